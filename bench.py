@@ -1,0 +1,605 @@
+"""Benchmark of the SAGA + Atop-N decode attention step on B200.
+
+One step = one decode token through the workload's attention stack: for every
+layer, either a plain Atop-N step (saga_decode_step) or, when t mod R == 0, a
+refresh (saga_refresh_threshold with V and out, which also runs that step).
+The default workload is the Llama-3.2-1B-shaped 16-layer stack at batch 8 and
+128K context (h_q=32, h_k=2, h_v=8, d=64, bf16 caches, N=2048, R=32).
+
+Prints one JSON line (rank 0):
+  value      steps/s of the whole job, inputs resident in HBM (CUDA events
+             over exactly --steps steps, max over ranks);
+  e2e        the same metric with queries copied in from pinned host memory
+             and outputs read back every step;
+  roofline   the plain-step call (the dominant one): algorithmic bytes per
+             call / its mean duration, against the measured HBM copy peak;
+  dense_gqa  the library's dense GQA stack at the same shape, same metric;
+  cpu_baseline  the float64 oracle on the host cores, on a bounded sample.
+
+With --impl reference the oracle alone is timed (the reference arm).
+Multi-GPU (torchrun): every rank runs its own batch (weak scaling), no
+collective on the data path.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+DEFAULT_WORKLOAD = "llama1b_stack16_b8_128k"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+METRIC = "SAGA+Atop-N decode-attn steps/s at 128K ctx; HBM GB/s vs peak"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--dense-steps", type=int, default=8)
+    ap.add_argument("--layers", type=int, default=None,
+                    help="override the stack depth (same per-layer launch, smaller footprint)")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+def dist_init():
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# measurement helpers
+# ---------------------------------------------------------------------------
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(smax)),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def source_hash(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_sources):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    if d.get("source_hash") != source_hash(kernel_sources):
+        return None
+    return d.get("dram_bytes_per_call")
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host cores (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+class OracleSample:
+    """One (sequence, key-head group) of one layer, the bounded sample the
+    oracle is timed on; scaled by the number of such groups per step."""
+
+    def __init__(self, w):
+        self.w = w
+        L = int(synth.seq_lens(w)[0])
+        G = w.h_q // w.h_k
+        hv_g = w.h_v // w.h_k
+        self.L, self.G = L, G
+        self.groups_per_step = w.layers * w.B * w.h_k
+        K = synth.widen(synth.cache_rows(w, 0, "K", 0, 0, 0, L))
+        V = np.stack([synth.widen(synth.cache_rows(w, 0, "V", 0, v, 0, L)) for v in range(hv_g)])
+        self.K = K[None, None]             # [1][1][L][d]
+        self.V = V[None]                   # [1][hv_g][L][d]
+        self.l = np.array([L])
+        steps = max(2, 2)
+        qs = synth.widen(synth.queries(w, 0, steps, B=1, h_q=G))
+        self.qs = qs                       # [steps][1][G][d]
+        self.tau = None
+
+    def step(self, t, refresh):
+        import oracle
+        q = self.qs[t % len(self.qs)]
+        if refresh or self.tau is None:
+            self.tau = oracle.refresh(q, self.K, self.l, self.w.N)
+        oracle.decode_step(q, self.K, self.V, self.l, self.tau)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def time_oracle(w, n_plain=2, n_refresh=1):
+    """Seconds per full step (every layer, sequence and key-head group), from
+    timing the sample's plain and refresh steps."""
+    s = OracleSample(w)
+    s.step(0, True)                                   # warm
+    t0 = time.perf_counter()
+    for i in range(n_refresh):
+        s.step(i, True)
+    t_ref = (time.perf_counter() - t0) / n_refresh
+    t0 = time.perf_counter()
+    for i in range(n_plain):
+        s.step(i + 1, False)
+    t_plain = (time.perf_counter() - t0) / n_plain
+    per_group = (t_ref + (w.R - 1) * t_plain) / w.R
+    return per_group * s.groups_per_step, t_plain, t_ref, s
+
+
+def reference_arm(args, w):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    s = OracleSample(w)
+    for t in range(args.warmup):
+        s.step(t, t % w.R == 0)
+    t0 = time.perf_counter()
+    for t in range(args.warmup, args.warmup + args.steps):
+        s.step(t, t % w.R == 0)
+    sample_s = time.perf_counter() - t0
+    step_s = sample_s / args.steps * s.groups_per_step
+    v = 1.0 / step_s
+    sample = (f"layer 0, sequence 0, key head 0 ({s.G} query heads, l_kv={s.L}) of each "
+              f"step, scaled by {s.groups_per_step} groups per step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "steps/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, world),
+        "cpu_baseline": {"value": v, "unit": "steps/s", "cores": blas_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w, world):
+    return {"workload": w.name, "batch_per_gpu": w.B, "global_batch": w.B * world,
+            "layers": w.layers, "h_q": w.h_q, "h_k": w.h_k, "h_v": w.h_v, "d": w.d,
+            "l_kv": w.l_kv if w.l_kv_range is None else list(w.l_kv_range), "N": w.N,
+            "R": w.R, "dense_gqa_h_kv": w.dense_hkv,
+            "parallelism": f"weak: {world} independent batch replica(s)"}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+class Stack:
+    """Device state of one attention stack: per-layer caches, thresholds,
+    outputs, the static query buffer and the workspace."""
+
+    def __init__(self, w, saga, dense=False):
+        import torch
+        from synth import device as sdev
+        self.w, self.dense = w, dense
+        h_k = w.dense_hkv if dense else w.h_k
+        h_v = w.dense_hkv if dense else w.h_v
+        kk, vk = ("KD", "VD") if dense else ("K", "V")
+        self.lens = synth.seq_lens(w)
+        cap = int(self.lens.max())
+        self.cap = cap
+        self.shape = saga.shape(w.B, w.h_q, h_k, h_v, w.d, w.dtype, cap, cap)
+        esz = w.elem_bytes
+        layer_bytes = w.B * (h_k + h_v) * cap * w.d * esz
+        # single-layer workloads rotate bit-identical replicas so the working
+        # set stays well above L2
+        self.replicas = 1 if w.layers > 1 else max(1, math.ceil(4 * L2_BYTES / layer_bytes))
+        self.nl = w.layers
+        dt = torch.float32 if w.dtype == synth.F32 else torch.int16
+        self.K, self.V = [], []
+        for r in range(self.replicas):
+            for l in range(self.nl):
+                if r == 0:
+                    K = torch.empty(w.B, h_k, cap, w.d, dtype=dt, device="cuda")
+                    V = torch.empty(w.B, h_v, cap, w.d, dtype=dt, device="cuda")
+                    sdev.fill(K, w, l, kk)
+                    sdev.fill(V, w, l, vk)
+                else:
+                    K = self.K[l].clone()
+                    V = self.V[l].clone()
+                self.K.append(K)
+                self.V.append(V)
+        self.l = torch.from_numpy(self.lens).cuda()
+        self.tau = torch.zeros(self.nl, w.B, w.h_q, dtype=torch.float32, device="cuda")
+        self.out = torch.zeros(self.nl, w.B, w.h_q, w.d, dtype=torch.float32, device="cuda")
+        self.q = torch.zeros(self.nl, w.B, w.h_q, w.d, dtype=dt, device="cuda")
+        self.ws = saga.Workspace(self.shape, w.N)
+        self.saga = saga
+
+    def layer_call(self, t, l, refresh, sel_mask=None):
+        r = t % self.replicas
+        K, V = self.K[r * self.nl + l], self.V[r * self.nl + l]
+        s = self.saga
+        if self.dense:
+            s.gqa_dense_decode(self.shape, self.q[l], K, V, self.l, self.out[l], self.ws)
+        elif refresh:
+            s.refresh_threshold(self.shape, self.q[l], K, self.l, self.w.N, self.tau[l], self.ws,
+                                V=V, out=self.out[l], sel_mask=sel_mask)
+        else:
+            s.decode_step(self.shape, self.q[l], K, V, self.l, self.tau[l], self.out[l], self.ws,
+                          sel_mask=sel_mask)
+
+    def step(self, t, refresh):
+        for l in range(self.nl):
+            self.layer_call(t, l, refresh)
+
+
+def kernels_per_call(dense, refresh):
+    if dense:
+        return 2                  # dense split + combine
+    return 4 if refresh else 2    # (dump, radix,) split + combine
+
+
+def run_ours(args, w):
+    import torch
+    import sparse_decode_attention_step_b200 as saga
+    saga.load()
+    world, rank, local = dist_init()
+    if world > 1:
+        w = w.with_(seed=w.seed + 7919 * rank)
+    torch.manual_seed(0)
+    R = w.R
+    T_total = args.warmup + args.steps
+    st = Stack(w, saga)
+    esz = w.elem_bytes
+    # queries of every step, resident in HBM, and their pinned host copies
+    qh = np.stack([synth.queries(w, l, T_total) for l in range(w.layers)], axis=1)
+    if w.dtype != synth.F32:
+        qh = qh.view(np.int16)
+    Q = torch.from_numpy(qh).cuda()                     # [T][layers][B][h_q][d]
+    Qpin = torch.from_numpy(qh).pin_memory()
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream()
+
+    def enqueue(t):
+        st.q.copy_(Q[t], non_blocking=True)
+        st.step(t, t % R == 0)
+
+    def capture(t0, t1):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for t in range(t0, t1):
+                enqueue(t)
+        return g
+
+    # warm-up steps run directly (they load every kernel before any capture)
+    for t in range(args.warmup):
+        enqueue(t)
+    torch.cuda.synchronize()
+    use_graph = not args.no_graph
+    if use_graph:
+        g_timed = capture(args.warmup, T_total)
+        torch.cuda.synchronize()
+    barrier(world)
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        time.sleep(0.3)
+        torch.cuda.synchronize()
+        barrier(world)
+        if not use_graph:
+            torch.cuda._sleep(int(2e8))      # let the host run ahead of the GPU
+        ev0.record(stream)
+        if use_graph:
+            g_timed.replay()
+        else:
+            for t in range(args.warmup, T_total):
+                enqueue(t)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    elapsed_ms = ev0.elapsed_time(ev1)
+    max_ms = max_over_ranks(elapsed_ms, world)
+    value = world * args.steps / (max_ms / 1e3)
+    n_refresh = sum(1 for t in range(args.warmup, T_total) if t % R == 0)
+    launches = w.layers * (n_refresh * kernels_per_call(False, True)
+                           + (args.steps - n_refresh) * kernels_per_call(False, False))
+    if use_graph:
+        del g_timed
+
+    # ---- roofline: per-call durations of plain steps, and algorithmic bytes
+    # from a validation pass with the selection dumped
+    torch.cuda.synchronize()
+    evs = []
+    n_rl = min(args.steps, 2 * R)
+    torch.cuda._sleep(int(4e8))              # let the host run ahead of the GPU
+    for t in range(args.warmup, args.warmup + n_rl):
+        st.q.copy_(Q[t])
+        refresh = t % R == 0
+        for l in range(w.layers):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            st.layer_call(t, l, refresh)
+            b.record(stream)
+            evs.append((refresh, a, b))
+    torch.cuda.synchronize()
+    plain_ms = [a.elapsed_time(b) for (r, a, b) in evs if not r]
+    refresh_ms = [a.elapsed_time(b) for (r, a, b) in evs if r]
+    call_ms = float(np.mean(plain_ms)) if plain_ms else float("nan")
+    refresh_call_ms = float(np.mean(refresh_ms)) if refresh_ms else None
+
+    B, h_q, h_k, h_v, d = w.B, w.h_q, w.h_k, w.h_v, w.d
+    lens = st.lens.astype(np.int64)
+    k_bytes = float(np.sum(h_k * lens * d * esz))
+    qo_bytes = B * h_q * d * (esz + 4) + B * h_q * 4
+    mask = torch.zeros(B, h_q, st.cap, dtype=torch.uint8, device="cuda")
+    v_bytes, v_bytes_nodedup = [], []
+    for t in range(args.warmup, args.warmup + min(args.steps, 2 * R)):
+        st.q.copy_(Q[t])
+        refresh = t % R == 0
+        for l in range(w.layers):
+            mask.zero_()
+            st.layer_call(t, l, refresh, sel_mask=mask)
+            if refresh:
+                continue
+            m = mask.view(B, h_v, h_q // h_v, st.cap)
+            distinct = int(m.amax(dim=2).sum().item())
+            v_bytes.append(distinct * d * esz)
+            v_bytes_nodedup.append(int(mask.sum().item()) * d * esz)
+    torch.cuda.synchronize()
+    alg_bytes = k_bytes + float(np.mean(v_bytes)) + qo_bytes
+    achieved = alg_bytes / (call_ms / 1e3) / 1e9
+    peak, peak_kind = measured_peaks()
+    here = os.path.join(ROOT, "sparse_decode_attention_step_b200", "csrc")
+    ksrc = [os.path.join(here, f) for f in sorted(os.listdir(here))]
+    traffic = ncu_traffic(ksrc)
+
+    # ---- e2e: queries in from pinned host memory, outputs back, every step
+    out_pin = torch.empty(st.out.shape, dtype=torch.float32).pin_memory()
+    l_pin = torch.from_numpy(st.lens).pin_memory()
+    graphs = {}
+    if use_graph:
+        for r in range(st.replicas):
+            for kind in (True, False):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    st.step(r, kind)
+                graphs[(kind, r)] = g
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for t in range(args.warmup, T_total):
+        st.q.copy_(Qpin[t], non_blocking=True)
+        st.l.copy_(l_pin, non_blocking=True)
+        refresh = t % R == 0
+        if graphs:
+            graphs[(refresh, t % st.replicas)].replay()
+        else:
+            st.step(t, refresh)
+        out_pin.copy_(st.out, non_blocking=True)
+        stream.synchronize()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_value = world * args.steps / (e2e_ms / 1e3)
+    h2d = Q[0].numel() * Q.element_size() + l_pin.numel() * 4
+    d2h = st.out.numel() * 4
+
+    # ---- dense GQA stack at the same shape
+    dense = None
+    if not args.no_dense and w.dense_hkv is not None:
+        del graphs
+        stk_dense = Stack(w, saga, dense=True)
+        stk_dense.q.copy_(Q[0])
+        for t in range(2):
+            stk_dense.step(t, False)
+        torch.cuda.synchronize()
+        barrier(world)
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        nd = args.dense_steps
+
+        def dense_steps():
+            for t in range(nd):
+                stk_dense.q.copy_(Q[t % T_total], non_blocking=True)
+                stk_dense.step(t, False)
+        if use_graph:
+            gd = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gd):
+                dense_steps()
+            torch.cuda.synchronize()
+        else:
+            torch.cuda._sleep(int(2e8))
+        d0.record(stream)
+        if use_graph:
+            gd.replay()
+        else:
+            dense_steps()
+        d1.record(stream)
+        torch.cuda.synchronize()
+        dms = max_over_ranks(d0.elapsed_time(d1), world)
+        dvalue = world * nd / (dms / 1e3)
+        dbytes_step = w.layers * (2 * w.dense_hkv * float(np.sum(lens)) * d * esz + qo_bytes)
+        dgbs = dbytes_step / (dms / nd / 1e3) / 1e9
+        dense = {"value": dvalue, "unit": "steps/s", "ms_per_step": dms / nd,
+                 "tokens_per_s": dvalue * B, "achieved_gbs": dgbs, "frac_of_peak": dgbs / peak,
+                 "h_kv": w.dense_hkv, "steps": nd, "speedup_saga_over_dense": value / dvalue}
+        del stk_dense
+        torch.cuda.empty_cache()
+
+    clocks = clk.summary()
+    result = None
+    if rank == 0:
+        cpu = None
+        if not args.no_cpu_baseline:
+            step_s, t_plain, t_ref, s = time_oracle(w)
+            cpu = {"value": 1.0 / step_s, "unit": "steps/s", "cores": blas_threads(),
+                   "kind": "oracle",
+                   "sample": (f"layer 0, sequence 0, key head 0 ({s.G} query heads, "
+                              f"l_kv={s.L}): 1 refresh + 2 plain steps timed, R-cycle "
+                              f"average, scaled by {s.groups_per_step} groups per step"),
+                   "sample_plain_s": t_plain, "sample_refresh_s": t_ref}
+        result = {
+            "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype != synth.F32 else "f32", "accumulate": "f32",
+            "data": "synthetic (seeded Philox N(0,1) K/V, 1% planted keys, AR(1) queries)",
+            "config": dict(workload_config(w, world),
+                           l2="inputs larger than L2" if st.replicas == 1 else
+                           f"{st.replicas} bit-identical cache replicas rotated",
+                           timed_region="one CUDA graph of all timed steps" if use_graph
+                           else "direct launches"),
+            "tokens_per_s": value * B,
+            "refresh_every": R, "refresh_steps_timed": n_refresh,
+            "gpu_launches": launches * world,
+            "roofline": {"bound": "hbm", "kernel": "saga_decode_step (split + combine)",
+                         "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_source": peak_kind,
+                         "traffic": traffic, "alg_bytes_per_call": alg_bytes,
+                         "call_ms": call_ms, "refresh_call_ms": refresh_call_ms,
+                         "v_bytes_per_call_distinct": float(np.mean(v_bytes)),
+                         "v_bytes_per_call_nodedup": float(np.mean(v_bytes_nodedup)),
+                         "frac_of_8000_nominal": achieved / 8000.0},
+            "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "dense_gqa": dense,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(result), flush=True)
+    barrier(world)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return result
+
+
+def main():
+    args = parse()
+    w = synth.WORKLOADS[args.workload]
+    if args.layers is not None:
+        w = w.with_(layers=args.layers)
+    if args.steps < 1 or args.warmup < 0:
+        raise SystemExit("--steps must be >= 1")
+    if args.impl == "reference":
+        reference_arm(args, w)
+        return
+    run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,185 @@
+/*
+ * saga.h -- C ABI of the SAGA + Atop-N single-token decode attention step
+ * on NVIDIA B200 (sm_100a).
+ *
+ * Source of the operations: "More Value per Key: Asymmetric Sparse Attention
+ * for Faster LLM Decoding" (the SAGA paper), as summarised on its pages:
+ *   - Attention Mechanism Formalization, Eq. (2-4): A = Q K^T / sqrt(d),
+ *     P = softmax(A), O = P V;
+ *   - Top-N Attention, Eq. (6): indices of the N largest entries per row;
+ *   - Methodology > Atop-N Attention, item 1: entries are kept by comparing
+ *     each score with a threshold equal to the N-th largest score; item 2:
+ *     the exact threshold is recomputed once every n tokens and reused;
+ *     Eq. (7): O = softmax(A[i]) V[i] over the kept entries only;
+ *   - SAGA Architecture: h_k key heads decoupled from h_v value heads
+ *     (h_k < h_v).
+ *
+ * One decode step, per sequence b and query head j (0 <= j < h_q):
+ *   A[b,j,t] = (q[b,j,:] . K[b, floor(j*h_k/h_q), t, :]) / sqrt(d),  t < l_kv[b]
+ *   S[b,j]   = { t : A[b,j,t] >= tau[b,j] }
+ *   out[b,j] = sum_{t in S} e^{A[b,j,t]-m} V[b, floor(j*h_v/h_q), t, :]
+ *              / sum_{t in S} e^{A[b,j,t]-m},   m = max_{t in S} A[b,j,t]
+ *   out[b,j] = 0 when S is empty.
+ * A refresh sets tau[b,j] to the exact N-th largest A[b,j,:] (under IEEE
+ * totalOrder of the fp32 scores, so it is always one of them), or to -inf
+ * when N >= l_kv[b] (every entry kept).
+ *
+ * Conventions for every call:
+ *   - All array pointers are DEVICE pointers, owned by the caller. The
+ *     library allocates nothing and keeps no global mutable state; calls
+ *     that use distinct workspaces may run concurrently.
+ *   - Every call is asynchronous on `stream` (NULL = the legacy default
+ *     stream) and returns after enqueueing its kernels. A returned error
+ *     means nothing was enqueued, except SAGA_ERR_CUDA, which means a launch
+ *     failed.
+ *   - Arguments are checked on the host; a violation returns
+ *     SAGA_ERR_INVALID_ARG or SAGA_ERR_UNSUPPORTED and enqueues nothing.
+ *   - Per-sequence lengths are read on the device. A length outside
+ *     [0, min(cap, max_l_kv)] is clamped into that range and sets a bit in
+ *     the workspace's device error word (saga_read_device_error); kernels
+ *     never trap.
+ *   - Scores are computed in fp32 from the stored (fp32 or bf16) values;
+ *     every entry point computes a given score with the same arithmetic, so
+ *     a dumped score row is exactly the row the selection used.
+ */
+#ifndef SAGA_H_
+#define SAGA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same handle type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *saga_stream_t;
+
+typedef enum saga_status {
+  SAGA_OK = 0,
+  SAGA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size or shape */
+  SAGA_ERR_UNSUPPORTED = 2,  /* valid but outside what the kernels handle */
+  SAGA_ERR_WORKSPACE = 3,    /* workspace missing, misaligned or too small */
+  SAGA_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+  SAGA_ERR_DEVICE = 5        /* the device error word is non-zero */
+} saga_status;
+
+typedef enum saga_dtype {
+  SAGA_F32 = 0,   /* q, K, V stored as IEEE binary32 */
+  SAGA_BF16 = 1   /* q, K, V stored as bfloat16 */
+} saga_dtype;
+
+/* Device error word bits (saga_read_device_error). */
+#define SAGA_DEVERR_LKV_NEGATIVE 1   /* some l_kv[b] < 0, treated as 0 */
+#define SAGA_DEVERR_LKV_TOO_LONG 2   /* some l_kv[b] > min(cap, max_l_kv), clamped */
+
+/*
+ * Problem shape. Layouts (element strides, d contiguous within a row):
+ *   q   [B][h_q][d]       element (b,j,i)   at b*q_stride_b + j*q_stride_h + i
+ *   K   [B][h_k][cap][d]  element (b,h,t,i) at b*k_stride_b + h*k_stride_h + t*d + i
+ *   V   [B][h_v][cap][d]  element (b,h,t,i) at b*v_stride_b + h*v_stride_h + t*d + i
+ *   l_kv [B] int32, tau [B][h_q] fp32, out [B][h_q][d] fp32, all contiguous.
+ * Requirements: B >= 1; 1 <= h_k <= h_v <= h_q; h_q % h_v == 0;
+ * h_v % h_k == 0; h_q / h_k <= 16; d in {64, 128}; dtype a saga_dtype;
+ * 0 <= max_l_kv <= cap; every stride > 0 and a multiple of 16 bytes.
+ * max_l_kv is the host-side bound on every l_kv[b]; it sizes the work split
+ * and the workspace.
+ */
+typedef struct saga_shape {
+  int32_t B, h_q, h_k, h_v, d;
+  int32_t dtype;
+  int64_t cap;
+  int64_t max_l_kv;
+  int64_t q_stride_b, q_stride_h;
+  int64_t k_stride_b, k_stride_h;
+  int64_t v_stride_b, v_stride_h;
+} saga_shape;
+
+/* Fill `s` for contiguous q, K and V with the given sizes. */
+void saga_shape_contiguous(saga_shape *s, int32_t B, int32_t h_q, int32_t h_k,
+                           int32_t h_v, int32_t d, int32_t dtype, int64_t cap,
+                           int64_t max_l_kv);
+
+/*
+ * Bytes of device workspace that saga_decode_step, saga_refresh_threshold
+ * (with this N) and gqa_dense_decode need for `shape`; 0 if the shape is
+ * invalid. The workspace must be 256-byte aligned, must be passed to
+ * saga_workspace_init once after allocation, and must not be used by two
+ * calls that run concurrently. It holds the device error word, per-split
+ * partial softmax states and, for refresh, one fp32 score row per
+ * (sequence, query head).
+ */
+size_t saga_workspace_size(const saga_shape *shape, int32_t N);
+
+/* Zero a newly allocated workspace (asynchronous on `stream`). */
+saga_status saga_workspace_init(void *ws, size_t ws_bytes, saga_stream_t stream);
+
+/*
+ * One plain Atop-N step with stored thresholds (Atop-N item 1 and Eq. 7).
+ *   q, K, V   inputs as described by `shape`.
+ *   l_kv      [B] int32, valid positions per sequence.
+ *   tau       [B][h_q] fp32 thresholds, read only.
+ *   out       [B][h_q][d] fp32, written.
+ *   sel_count nullable [B][h_q] int32: receives |S[b,j]|.
+ *   sel_mask  nullable [B][h_q][max_l_kv] uint8: entry t < l_kv[b] receives
+ *             1 if t was kept, else 0; entries t >= l_kv[b] are not written.
+ */
+saga_status saga_decode_step(const saga_shape *shape, const void *q,
+                             const void *K, const void *V,
+                             const int32_t *l_kv, const float *tau,
+                             float *out, int32_t *sel_count,
+                             uint8_t *sel_mask, void *ws, size_t ws_bytes,
+                             saga_stream_t stream);
+
+/*
+ * Refresh step (Atop-N item 2): tau[b][j] = the exact N-th largest score of
+ * row (b, j) under IEEE totalOrder, or -inf when N >= l_kv[b]. N >= 1.
+ *   V, out    both NULL: only tau is written. Both non-NULL: the same call
+ *             then runs this step's selection and PV with the fresh tau,
+ *             exactly as saga_decode_step would (out, sel_count, sel_mask as
+ *             there). One NULL and the other not: SAGA_ERR_INVALID_ARG.
+ *   scores    nullable [B][h_q][max_l_kv] fp32: receives the score rows the
+ *             thresholds were selected from (entries t < l_kv[b]).
+ */
+saga_status saga_refresh_threshold(const saga_shape *shape, const void *q,
+                                   const void *K, const void *V,
+                                   const int32_t *l_kv, int32_t N,
+                                   float *tau, float *out,
+                                   int32_t *sel_count, uint8_t *sel_mask,
+                                   float *scores, void *ws, size_t ws_bytes,
+                                   saga_stream_t stream);
+
+/*
+ * Full-attention GQA decode (Eq. 2-4 over every t < l_kv[b]): the dense
+ * baseline the sparse step is measured against. Requires h_k == h_v.
+ */
+saga_status gqa_dense_decode(const saga_shape *shape, const void *q,
+                             const void *K, const void *V,
+                             const int32_t *l_kv, float *out, void *ws,
+                             size_t ws_bytes, saga_stream_t stream);
+
+/*
+ * Write the fp32 score rows A[b][j][t], t < l_kv[b], into
+ * scores [B][h_q][max_l_kv], with the same arithmetic as every other entry
+ * point. For checking. Uses the workspace's error word only.
+ */
+saga_status saga_debug_scores(const saga_shape *shape, const void *q,
+                              const void *K, const int32_t *l_kv,
+                              float *scores, void *ws, size_t ws_bytes,
+                              saga_stream_t stream);
+
+/*
+ * Synchronise `stream`, copy the device error word to *flags and clear it.
+ * Returns SAGA_ERR_DEVICE if it was non-zero, SAGA_OK otherwise.
+ */
+saga_status saga_read_device_error(void *ws, saga_stream_t stream,
+                                   int32_t *flags);
+
+/* Static description of a status code. */
+const char *saga_status_string(saga_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAGA_H_ */

@@ -1,0 +1,217 @@
+// Dense GQA decode split kernel: the full-attention baseline, Eq. (2-4) over
+// every position. One CTA per (b, kv head, split of l_kv). Each sub-chunk of
+// 256 positions is scored (one position per thread, all G query heads of the
+// group), the chunk maximum updates the running softmax state, and the
+// probabilities weight the V rows (one V row per warp-iteration, d split
+// across the lanes). The per-split states go to the same combine kernel as
+// the sparse step.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace saga {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kChunk = kThreads;
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <typename T, int D, int GP>
+__device__ __forceinline__ void dense_scores(const T *krow, const float *qs, float scale,
+                                             float (&A)[GP]) {
+  float acc[GP];
+#pragma unroll
+  for (int g = 0; g < GP; ++g) acc[g] = 0.f;
+#pragma unroll 2
+  for (int c = 0; c < D; c += 8) {
+    float k[8];
+    load8(krow + c, k);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float4 *qv = reinterpret_cast<const float4 *>(qs + (c + e) * GP);
+#pragma unroll
+      for (int g4 = 0; g4 < GP / 4; ++g4) {
+        float4 w = qv[g4];
+        acc[4 * g4 + 0] = fmaf(w.x, k[e], acc[4 * g4 + 0]);
+        acc[4 * g4 + 1] = fmaf(w.y, k[e], acc[4 * g4 + 1]);
+        acc[4 * g4 + 2] = fmaf(w.z, k[e], acc[4 * g4 + 2]);
+        acc[4 * g4 + 3] = fmaf(w.w, k[e], acc[4 * g4 + 3]);
+      }
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < GP; ++g) A[g] = acc[g] * scale;
+}
+
+__device__ __forceinline__ float widen1(const float *p) { return *p; }
+__device__ __forceinline__ float widen1(const uint16_t *p) {
+  return __uint_as_float(static_cast<uint32_t>(*p) << 16);
+}
+
+template <int VPL>
+__device__ __forceinline__ void vslice(const float *row, int lane, float (&v)[VPL]) {
+  if constexpr (VPL == 2) {
+    float2 a = __ldg(reinterpret_cast<const float2 *>(row) + lane);
+    v[0] = a.x; v[1] = a.y;
+  } else {
+    float4 a = __ldg(reinterpret_cast<const float4 *>(row) + lane);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  }
+}
+template <int VPL>
+__device__ __forceinline__ void vslice(const uint16_t *row, int lane, float (&v)[VPL]) {
+  if constexpr (VPL == 2) {
+    uint32_t a = __ldg(reinterpret_cast<const uint32_t *>(row) + lane);
+    v[0] = bf16lo(a); v[1] = bf16hi(a);
+  } else {
+    uint2 a = __ldg(reinterpret_cast<const uint2 *>(row) + lane);
+    v[0] = bf16lo(a.x); v[1] = bf16hi(a.x); v[2] = bf16lo(a.y); v[3] = bf16hi(a.y);
+  }
+}
+
+template <typename T, int D, int GP>
+__global__ void __launch_bounds__(kThreads) dense_split_kernel(const StepParams p) {
+  constexpr int VPL = D / 32;
+  __shared__ __align__(16) float qs[D * GP];
+  __shared__ __align__(16) float ps[kChunk][GP];
+  __shared__ float red[kWarps][GP];
+  __shared__ float red_acc[kWarps][GP][D];
+  __shared__ float red_l[kWarps][GP];
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int s = blockIdx.x;
+  const int b = blockIdx.y / p.h_k, kh = blockIdx.y % p.h_k;
+  const int G = p.h_q / p.h_k;
+  const int j0 = kh * G;
+  const int64_t L = clamp_len(p, b);
+  const int64_t t_begin = static_cast<int64_t>(s) * p.split_len;
+  if (t_begin >= L) return;
+  const int64_t t_end = min(t_begin + p.split_len, L);
+
+  const T *qg = static_cast<const T *>(p.q) + b * p.q_sb;
+  for (int idx = tid; idx < D * GP; idx += kThreads) {
+    int i = idx / GP, g = idx % GP;
+    qs[idx] = g < G ? widen1(qg + (j0 + g) * p.q_sh + i) : 0.f;
+  }
+  __syncthreads();
+
+  const T *krow0 = static_cast<const T *>(p.K) + b * p.k_sb + kh * p.k_sh;
+  const T *vrow0 = static_cast<const T *>(p.V) + b * p.v_sb + kh * p.v_sh;
+
+  float m_run[GP], l_run[GP], acc[GP][VPL];
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+    m_run[g] = -INFINITY; l_run[g] = 0.f;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) acc[g][v] = 0.f;
+  }
+
+  for (int64_t base = t_begin; base < t_end; base += kChunk) {
+    const int64_t t = base + tid;
+    const bool valid = t < t_end;
+    float A[GP];
+    if (valid) {
+      dense_scores<T, D, GP>(krow0 + t * D, qs, p.scale, A);
+    } else {
+#pragma unroll
+      for (int g = 0; g < GP; ++g) A[g] = -INFINITY;
+    }
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+      const float mx = warp_max(A[g]);
+      if (lane == 0) red[warp][g] = mx;
+    }
+    __syncthreads();
+    float m_new[GP];
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+      float mc = red[0][g];
+#pragma unroll
+      for (int w = 1; w < kWarps; ++w) mc = fmaxf(mc, red[w][g]);
+      m_new[g] = fmaxf(m_run[g], mc);
+      const float corr = exp2f((m_run[g] - m_new[g]) * kLog2e);
+      l_run[g] *= corr;
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) acc[g][v] *= corr;
+      m_run[g] = m_new[g];
+      ps[tid][g] = valid ? exp2f((A[g] - m_new[g]) * kLog2e) : 0.f;
+    }
+    __syncthreads();
+    const int n = static_cast<int>(t_end - base < kChunk ? t_end - base : kChunk);
+    for (int kk = warp; kk < n; kk += kWarps) {
+      float vv[VPL];
+      vslice<VPL>(vrow0 + (base + kk) * D, lane, vv);
+      const float4 *pv = reinterpret_cast<const float4 *>(&ps[kk][0]);
+#pragma unroll
+      for (int g4 = 0; g4 < GP / 4; ++g4) {
+        const float4 w = pv[g4];
+        const float pw[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          l_run[4 * g4 + u] += pw[u];
+#pragma unroll
+          for (int v = 0; v < VPL; ++v)
+            acc[4 * g4 + u][v] = fmaf(pw[u], vv[v], acc[4 * g4 + u][v]);
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+  // Every warp holds the same m_run; sum the warps' l and acc.
+  if (tid == 0) {
+#pragma unroll
+    for (int g = 0; g < GP; ++g) red[0][g] = m_run[g];
+  }
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) red_acc[warp][g][lane * VPL + v] = acc[g][v];
+    if (lane == 0) red_l[warp][g] = l_run[g];
+  }
+  __syncthreads();
+  for (int idx = tid; idx < G * D; idx += kThreads) {
+    const int g = idx / D, i = idx % D;
+    float a = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) a += red_acc[w][g][i];
+    float *rec = p.partials + (static_cast<int64_t>(b * p.h_q + j0 + g) * p.S + s) * (D + kRecPad);
+    rec[kRecPad + i] = a;
+    if (i == 0) {
+      float l = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) l += red_l[w][g];
+      rec[0] = red[0][g];
+      rec[1] = l;
+      rec[2] = __int_as_float(static_cast<int>(t_end - t_begin));
+      rec[3] = 0.f;
+    }
+  }
+}
+
+}  // namespace
+
+template <typename T, int D>
+static cudaError_t launch_dd(const StepParams &p, int gp, dim3 grid, cudaStream_t st) {
+  switch (gp) {
+    case 4: dense_split_kernel<T, D, 4><<<grid, kThreads, 0, st>>>(p); break;
+    case 8: dense_split_kernel<T, D, 8><<<grid, kThreads, 0, st>>>(p); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dense_split(const StepParams &p, int dtype, int d, int gp, cudaStream_t st) {
+  dim3 grid(p.S, p.B * p.h_k);
+  if (dtype == SAGA_BF16) {
+    if (d == 64) return launch_dd<uint16_t, 64>(p, gp, grid, st);
+    if (d == 128) return launch_dd<uint16_t, 128>(p, gp, grid, st);
+  } else {
+    if (d == 64) return launch_dd<float, 64>(p, gp, grid, st);
+    if (d == 128) return launch_dd<float, 128>(p, gp, grid, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace saga

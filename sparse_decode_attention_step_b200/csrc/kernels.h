@@ -1,0 +1,31 @@
+// Launchers of the SAGA kernels (host side, internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace saga {
+
+enum { kModeDump = 0, kModeStep = 1, kModeFromScores = 2 };
+
+// Split kernel over grid (S, B * h_k); gp = h_q / h_k rounded up to 4.
+cudaError_t launch_saga_split(const StepParams &p, int mode, int dtype, int d, int gp,
+                              cudaStream_t st);
+
+// Merge the per-split states of every (b, j) into out and sel_count.
+cudaError_t launch_combine(const float *partials, const int32_t *l_kv, int32_t *err,
+                           float *out, int32_t *sel_count, int B, int h_q, int d, int S,
+                           int64_t split_len, int64_t cap, int64_t max_l_kv,
+                           cudaStream_t st);
+
+// tau[b][j] = N-th largest of the stored score row (b, j), or -inf if N >= l_kv[b].
+cudaError_t launch_radix_select(const float *scores, int64_t row_stride, const int32_t *l_kv,
+                                int32_t *err, int N, float *tau, int B, int h_q, int64_t cap,
+                                int64_t max_l_kv, cudaStream_t st);
+
+// Dense GQA split kernel over grid (S, B * h_k), h_k == h_v; gp = h_q / h_k rounded up to 4.
+cudaError_t launch_dense_split(const StepParams &p, int dtype, int d, int gp, cudaStream_t st);
+
+}  // namespace saga

@@ -1,0 +1,258 @@
+// C ABI of the SAGA + Atop-N decode step: argument checks, the work plan
+// (split of l_kv across CTAs, workspace carve-up) and the kernel launches.
+// Nothing here allocates device memory or synchronises, except
+// saga_read_device_error, which synchronises by contract.
+#include <cmath>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "saga.h"
+
+namespace saga {
+namespace {
+
+constexpr int64_t kTargetCtas = 4 * 148;   // four resident CTAs per B200 SM
+constexpr int64_t kSplitQuantum = 256;     // split lengths are multiples of a sub-chunk
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+struct Plan {
+  int S;                    // splits per (b, key head)
+  int64_t split_len;        // positions per split
+  size_t off_partials, off_scores, total;
+};
+
+// Splits sized so the grid holds about kTargetCtas CTAs of equal length.
+Plan make_plan(const saga_shape &s) {
+  Plan p{};
+  const int64_t units = static_cast<int64_t>(s.B) * s.h_k;
+  const int64_t s_target = std::max<int64_t>(1, ceil_div(kTargetCtas, units));
+  const int64_t L = std::max<int64_t>(1, s.max_l_kv);
+  p.split_len = ceil_div(ceil_div(L, s_target), kSplitQuantum) * kSplitQuantum;
+  p.S = static_cast<int>(ceil_div(L, p.split_len));
+  const size_t rec = static_cast<size_t>(s.d + kRecPad) * sizeof(float);
+  p.off_partials = kAlign;   // [0, 256): device error word
+  p.off_scores = align_up(p.off_partials + static_cast<size_t>(s.B) * s.h_q * p.S * rec);
+  p.total = align_up(p.off_scores + static_cast<size_t>(s.B) * s.h_q * s.max_l_kv * sizeof(float));
+  return p;
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+saga_status check_shape(const saga_shape *s) {
+  if (s == nullptr) return SAGA_ERR_INVALID_ARG;
+  if (s->B < 1 || s->h_q < 1 || s->h_k < 1 || s->h_v < 1 || s->d < 1) return SAGA_ERR_INVALID_ARG;
+  if (s->h_k > s->h_v || s->h_v > s->h_q) return SAGA_ERR_INVALID_ARG;
+  if (s->dtype != SAGA_F32 && s->dtype != SAGA_BF16) return SAGA_ERR_INVALID_ARG;
+  if (s->max_l_kv < 0 || s->cap < s->max_l_kv) return SAGA_ERR_INVALID_ARG;
+  if (s->h_q % s->h_v != 0 || s->h_v % s->h_k != 0) return SAGA_ERR_UNSUPPORTED;
+  if (s->h_q / s->h_k > kMaxGroup) return SAGA_ERR_UNSUPPORTED;
+  if (s->d != 64 && s->d != 128) return SAGA_ERR_UNSUPPORTED;
+  if (s->max_l_kv > INT32_MAX) return SAGA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(s->B) * s->h_k > 65535) return SAGA_ERR_UNSUPPORTED;
+  const int64_t esz = s->dtype == SAGA_F32 ? 4 : 2;
+  const int64_t st[6] = {s->q_stride_b, s->q_stride_h, s->k_stride_b,
+                         s->k_stride_h, s->v_stride_b, s->v_stride_h};
+  for (int64_t x : st)
+    if (x <= 0 || (x * esz) % 16 != 0) return SAGA_ERR_INVALID_ARG;
+  if (s->q_stride_h < s->d || s->k_stride_h < s->cap * s->d || s->v_stride_h < s->cap * s->d)
+    return SAGA_ERR_INVALID_ARG;
+  return SAGA_OK;
+}
+
+saga_status check_ws(const saga_shape &s, void *ws, size_t ws_bytes) {
+  if (ws == nullptr || !aligned(ws, kAlign)) return SAGA_ERR_WORKSPACE;
+  if (ws_bytes < make_plan(s).total) return SAGA_ERR_WORKSPACE;
+  return SAGA_OK;
+}
+
+saga_status check_inputs(const saga_shape &s, const void *q, const void *K, const int32_t *l_kv) {
+  if (q == nullptr || K == nullptr || l_kv == nullptr) return SAGA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(K, 16) || !aligned(l_kv, 4)) return SAGA_ERR_INVALID_ARG;
+  (void)s;
+  return SAGA_OK;
+}
+
+StepParams base_params(const saga_shape &s, const Plan &pl, const void *q, const void *K,
+                       const void *V, const int32_t *l_kv, void *ws) {
+  StepParams p{};
+  p.q = q; p.K = K; p.V = V; p.l_kv = l_kv;
+  p.err = static_cast<int32_t *>(ws);
+  p.partials = reinterpret_cast<float *>(static_cast<char *>(ws) + pl.off_partials);
+  p.q_sb = s.q_stride_b; p.q_sh = s.q_stride_h;
+  p.k_sb = s.k_stride_b; p.k_sh = s.k_stride_h;
+  p.v_sb = s.v_stride_b; p.v_sh = s.v_stride_h;
+  p.cap = s.cap; p.max_l_kv = s.max_l_kv; p.row_stride = s.max_l_kv;
+  p.split_len = pl.split_len;
+  p.B = s.B; p.h_q = s.h_q; p.h_k = s.h_k; p.h_v = s.h_v; p.S = pl.S;
+  p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(s.d)));
+  return p;
+}
+
+int group_pad(const saga_shape &s) { return ((s.h_q / s.h_k) + 3) / 4 * 4; }
+
+saga_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SAGA_OK : SAGA_ERR_CUDA; }
+
+// Select + PV over the stored thresholds, then the combine.
+saga_status run_step(const saga_shape &s, const Plan &pl, StepParams p, int mode,
+                     float *out, int32_t *sel_count, cudaStream_t st) {
+  cudaError_t e = launch_saga_split(p, mode, s.dtype, s.d, group_pad(s), st);
+  if (e != cudaSuccess) return SAGA_ERR_CUDA;
+  e = launch_combine(p.partials, p.l_kv, p.err, out, sel_count, s.B, s.h_q, s.d, pl.S,
+                     pl.split_len, s.cap, s.max_l_kv, st);
+  return cuda_status(e);
+}
+
+}  // namespace
+}  // namespace saga
+
+using namespace saga;
+
+extern "C" {
+
+void saga_shape_contiguous(saga_shape *s, int32_t B, int32_t h_q, int32_t h_k, int32_t h_v,
+                           int32_t d, int32_t dtype, int64_t cap, int64_t max_l_kv) {
+  if (s == nullptr) return;
+  std::memset(s, 0, sizeof(*s));
+  s->B = B; s->h_q = h_q; s->h_k = h_k; s->h_v = h_v; s->d = d; s->dtype = dtype;
+  s->cap = cap; s->max_l_kv = max_l_kv;
+  s->q_stride_h = d; s->q_stride_b = static_cast<int64_t>(h_q) * d;
+  s->k_stride_h = cap * d; s->k_stride_b = static_cast<int64_t>(h_k) * cap * d;
+  s->v_stride_h = cap * d; s->v_stride_b = static_cast<int64_t>(h_v) * cap * d;
+}
+
+size_t saga_workspace_size(const saga_shape *shape, int32_t N) {
+  (void)N;
+  if (check_shape(shape) != SAGA_OK) return 0;
+  return make_plan(*shape).total;
+}
+
+saga_status saga_workspace_init(void *ws, size_t ws_bytes, saga_stream_t stream) {
+  if (ws == nullptr || !aligned(ws, kAlign) || ws_bytes < kAlign) return SAGA_ERR_WORKSPACE;
+  return cuda_status(cudaMemsetAsync(ws, 0, kAlign, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+saga_status saga_decode_step(const saga_shape *shape, const void *q, const void *K,
+                             const void *V, const int32_t *l_kv, const float *tau, float *out,
+                             int32_t *sel_count, uint8_t *sel_mask, void *ws, size_t ws_bytes,
+                             saga_stream_t stream) {
+  saga_status r = check_shape(shape);
+  if (r != SAGA_OK) return r;
+  const saga_shape &s = *shape;
+  if ((r = check_inputs(s, q, K, l_kv)) != SAGA_OK) return r;
+  if (V == nullptr || !aligned(V, 16) || tau == nullptr || out == nullptr ||
+      !aligned(tau, 4) || !aligned(out, 16) || (sel_count && !aligned(sel_count, 4)))
+    return SAGA_ERR_INVALID_ARG;
+  if ((r = check_ws(s, ws, ws_bytes)) != SAGA_OK) return r;
+  const Plan pl = make_plan(s);
+  StepParams p = base_params(s, pl, q, K, V, l_kv, ws);
+  p.tau = tau;
+  p.sel_mask = sel_mask;
+  return run_step(s, pl, p, kModeStep, out, sel_count, reinterpret_cast<cudaStream_t>(stream));
+}
+
+saga_status saga_refresh_threshold(const saga_shape *shape, const void *q, const void *K,
+                                   const void *V, const int32_t *l_kv, int32_t N, float *tau,
+                                   float *out, int32_t *sel_count, uint8_t *sel_mask,
+                                   float *scores, void *ws, size_t ws_bytes,
+                                   saga_stream_t stream) {
+  saga_status r = check_shape(shape);
+  if (r != SAGA_OK) return r;
+  const saga_shape &s = *shape;
+  if ((r = check_inputs(s, q, K, l_kv)) != SAGA_OK) return r;
+  if (N < 1 || tau == nullptr || !aligned(tau, 4)) return SAGA_ERR_INVALID_ARG;
+  if ((V == nullptr) != (out == nullptr)) return SAGA_ERR_INVALID_ARG;
+  if (V != nullptr && (!aligned(V, 16) || !aligned(out, 16))) return SAGA_ERR_INVALID_ARG;
+  if ((scores && !aligned(scores, 4)) || (sel_count && !aligned(sel_count, 4)))
+    return SAGA_ERR_INVALID_ARG;
+  if ((r = check_ws(s, ws, ws_bytes)) != SAGA_OK) return r;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const Plan pl = make_plan(s);
+  StepParams p = base_params(s, pl, q, K, V, l_kv, ws);
+  float *rows = scores != nullptr
+                    ? scores
+                    : reinterpret_cast<float *>(static_cast<char *>(ws) + pl.off_scores);
+  // 1. score rows
+  p.scores_out = rows;
+  cudaError_t e = launch_saga_split(p, kModeDump, s.dtype, s.d, group_pad(s), st);
+  if (e != cudaSuccess) return SAGA_ERR_CUDA;
+  // 2. exact N-th largest per row
+  e = launch_radix_select(rows, s.max_l_kv, l_kv, p.err, N, tau, s.B, s.h_q, s.cap, s.max_l_kv,
+                          st);
+  if (e != cudaSuccess) return SAGA_ERR_CUDA;
+  if (V == nullptr) return SAGA_OK;
+  // 3. this step's select + PV from the same rows, with the fresh tau
+  p.scores_out = nullptr;
+  p.scores_in = rows;
+  p.tau = tau;
+  p.sel_mask = sel_mask;
+  return run_step(s, pl, p, kModeFromScores, out, sel_count, st);
+}
+
+saga_status gqa_dense_decode(const saga_shape *shape, const void *q, const void *K,
+                             const void *V, const int32_t *l_kv, float *out, void *ws,
+                             size_t ws_bytes, saga_stream_t stream) {
+  saga_status r = check_shape(shape);
+  if (r != SAGA_OK) return r;
+  const saga_shape &s = *shape;
+  if (s.h_k != s.h_v) return SAGA_ERR_INVALID_ARG;
+  if (s.h_q / s.h_k > 8) return SAGA_ERR_UNSUPPORTED;
+  if ((r = check_inputs(s, q, K, l_kv)) != SAGA_OK) return r;
+  if (V == nullptr || !aligned(V, 16) || out == nullptr || !aligned(out, 16))
+    return SAGA_ERR_INVALID_ARG;
+  if ((r = check_ws(s, ws, ws_bytes)) != SAGA_OK) return r;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const Plan pl = make_plan(s);
+  StepParams p = base_params(s, pl, q, K, V, l_kv, ws);
+  cudaError_t e = launch_dense_split(p, s.dtype, s.d, group_pad(s), st);
+  if (e != cudaSuccess) return SAGA_ERR_CUDA;
+  e = launch_combine(p.partials, l_kv, p.err, out, nullptr, s.B, s.h_q, s.d, pl.S, pl.split_len,
+                     s.cap, s.max_l_kv, st);
+  return cuda_status(e);
+}
+
+saga_status saga_debug_scores(const saga_shape *shape, const void *q, const void *K,
+                              const int32_t *l_kv, float *scores, void *ws, size_t ws_bytes,
+                              saga_stream_t stream) {
+  saga_status r = check_shape(shape);
+  if (r != SAGA_OK) return r;
+  const saga_shape &s = *shape;
+  if ((r = check_inputs(s, q, K, l_kv)) != SAGA_OK) return r;
+  if (scores == nullptr || !aligned(scores, 4)) return SAGA_ERR_INVALID_ARG;
+  if (ws == nullptr || !aligned(ws, kAlign) || ws_bytes < kAlign) return SAGA_ERR_WORKSPACE;
+  const Plan pl = make_plan(s);
+  StepParams p = base_params(s, pl, q, K, nullptr, l_kv, ws);
+  p.partials = nullptr;
+  p.scores_out = scores;
+  return cuda_status(launch_saga_split(p, kModeDump, s.dtype, s.d, group_pad(s),
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+saga_status saga_read_device_error(void *ws, saga_stream_t stream, int32_t *flags) {
+  if (ws == nullptr || !aligned(ws, kAlign) || flags == nullptr) return SAGA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t h = 0;
+  if (cudaMemcpyAsync(&h, ws, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return SAGA_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, sizeof(int32_t), st) != cudaSuccess) return SAGA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SAGA_ERR_CUDA;
+  *flags = h;
+  return h != 0 ? SAGA_ERR_DEVICE : SAGA_OK;
+}
+
+const char *saga_status_string(saga_status status) {
+  switch (status) {
+    case SAGA_OK: return "ok";
+    case SAGA_ERR_INVALID_ARG: return "invalid argument";
+    case SAGA_ERR_UNSUPPORTED: return "unsupported shape or configuration";
+    case SAGA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case SAGA_ERR_CUDA: return "CUDA runtime or launch failure";
+    case SAGA_ERR_DEVICE: return "device error word set (out-of-contract input)";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

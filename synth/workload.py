@@ -220,3 +220,27 @@ def queries(w: Workload, layer, steps, B=None, h_q=None):
                 q = a * q + c * xi[t]
                 out[t, b, j] = to_storage(q, w.dtype)
     return out
+
+
+def cache_rows_at(w: Workload, layer, kind, b, head, ts):
+    """Storage values of cache rows at arbitrary positions ``ts`` of one
+    (b, head): shape [len(ts)][d]; identical to the same rows of cache_rows."""
+    tensor = {"K": T_K, "V": T_V, "KD": T_KD, "VD": T_VD}[kind]
+    ts = np.asarray(ts, dtype=np.int64)
+    d = w.d
+    if ts.size == 0:
+        return to_storage(np.zeros((0, d)), w.dtype)
+    blocks = (ts[:, None] * (d // 4) + np.arange(d // 4)[None, :]).reshape(-1)
+    w0, w1, w2, w3 = philox_words(w.seed, tensor, layer, b, head, blocks.astype(np.uint64))
+    z0, z1 = box_muller(w0, w1)
+    z2, z3 = box_muller(w2, w3)
+    z = np.stack([z0, z1, z2, z3], axis=1).reshape(ts.size, d)
+    if kind in ("K", "KD"):
+        plant_head = head if kind == "K" else 1000 + head
+        pw = philox_words(w.seed, T_PLANT, layer, b, plant_head, (ts // 4).astype(np.uint64))
+        words = np.stack(pw, axis=1)[np.arange(ts.size), ts % 4]
+        mask = words < np.uint32(PLANT_THRESH)
+        if mask.any():
+            u = unit_direction(w.seed, layer, d)
+            z[mask] = PLANT_SCALE * u[None, :] + PLANT_NOISE * z[mask]
+    return to_storage(z, w.dtype)
