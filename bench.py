@@ -61,18 +61,34 @@ def parse():
 # ---------------------------------------------------------------------------
 # distributed plumbing
 # ---------------------------------------------------------------------------
-def dist_init():
+def dist_init(backend=None):
+    """One process per GPU: NCCL over the node's GPUs (gloo for CPU-only
+    checks). Returns (world, rank, local_rank)."""
     import torch
     import torch.distributed as dist
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
+    if backend is None:
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+    if world > 1 and not dist.is_initialized():
         import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    torch.cuda.set_device(local)
+        kw = {"device_id": torch.device("cuda", local)} if backend == "nccl" else {}
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+    if backend == "nccl":
+        torch.cuda.set_device(local)
     return world, rank, local
+
+
+def _reduce(x, world, op):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=op)
+    return float(t.item())
 
 
 def barrier(world):
@@ -82,23 +98,25 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
-    if world == 1:
-        return x
-    import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return _reduce(x, world, dist.ReduceOp.MAX if world > 1 else None)
 
 
 def sum_over_ranks(x, world):
-    if world == 1:
-        return x
-    import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    return _reduce(x, world, dist.ReduceOp.SUM if world > 1 else None)
+
+
+def rank_workload(w, rank):
+    """Each rank decodes its own batch of the same workload (weak scaling):
+    rank 0 keeps the canonical seed, rank r > 0 draws independent inputs."""
+    return w if rank == 0 else w.with_(seed=w.seed + 7919 * rank)
+
+
+def aggregate_value(steps, max_ms, world):
+    """Whole-job steps/s: every rank ran `steps` steps of its own batch; the
+    job takes as long as the slowest rank."""
+    return world * steps / (max_ms / 1e3)
 
 
 # ---------------------------------------------------------------------------
@@ -357,8 +375,7 @@ def run_ours(args, w):
     import sparse_decode_attention_step_b200 as saga
     saga.load()
     world, rank, local = dist_init()
-    if world > 1:
-        w = w.with_(seed=w.seed + 7919 * rank)
+    w = rank_workload(w, rank)
     torch.manual_seed(0)
     R = w.R
     T_total = args.warmup + args.steps
@@ -413,7 +430,7 @@ def run_ours(args, w):
         barrier(world)
     elapsed_ms = ev0.elapsed_time(ev1)
     max_ms = max_over_ranks(elapsed_ms, world)
-    value = world * args.steps / (max_ms / 1e3)
+    value = aggregate_value(args.steps, max_ms, world)
     n_refresh = sum(1 for t in range(args.warmup, T_total) if t % R == 0)
     launches = w.layers * (n_refresh * kernels_per_call(False, True)
                            + (args.steps - n_refresh) * kernels_per_call(False, False))
@@ -495,7 +512,7 @@ def run_ours(args, w):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e_value = world * args.steps / (e2e_ms / 1e3)
+    e2e_value = aggregate_value(args.steps, e2e_ms, world)
     h2d = Q[0].numel() * Q.element_size() + l_pin.numel() * 4
     d2h = st.out.numel() * 4
 
@@ -531,7 +548,7 @@ def run_ours(args, w):
         d1.record(stream)
         torch.cuda.synchronize()
         dms = max_over_ranks(d0.elapsed_time(d1), world)
-        dvalue = world * nd / (dms / 1e3)
+        dvalue = aggregate_value(nd, dms, world)
         dbytes_step = w.layers * (2 * w.dense_hkv * float(np.sum(lens)) * d * esz + qo_bytes)
         dgbs = dbytes_step / (dms / nd / 1e3) / 1e9
         dense = {"value": dvalue, "unit": "steps/s", "ms_per_step": dms / nd,

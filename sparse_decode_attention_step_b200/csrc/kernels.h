@@ -14,6 +14,10 @@ enum { kModeDump = 0, kModeStep = 1, kModeFromScores = 2 };
 cudaError_t launch_saga_split(const StepParams &p, int mode, int dtype, int d, int gp,
                               cudaStream_t st);
 
+// Tensor-core split kernel (bf16 caches, d in {64, 128}, h_q/h_k <= 16):
+// dump and step modes, bit-identical scores between the two.
+cudaError_t launch_saga_tc(const StepParams &p, int mode, int d, int gp, cudaStream_t st);
+
 // Merge the per-split states of every (b, j) into out and sel_count.
 cudaError_t launch_combine(const float *partials, const int32_t *l_kv, int32_t *err,
                            float *out, int32_t *sel_count, int B, int h_q, int d, int S,

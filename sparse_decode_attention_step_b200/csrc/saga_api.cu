@@ -96,10 +96,19 @@ int group_pad(const saga_shape &s) { return ((s.h_q / s.h_k) + 3) / 4 * 4; }
 
 saga_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SAGA_OK : SAGA_ERR_CUDA; }
 
+// Score-producing modes (dump, step) go to the tensor-core kernel for bf16
+// caches (a failure there is reported, never replaced by another path); fp32
+// caches and the from-scores mode use the SIMT split kernel.
+cudaError_t launch_split(const saga_shape &s, const StepParams &p, int mode, cudaStream_t st) {
+  const int gp = group_pad(s);
+  if (mode != kModeFromScores && s.dtype == SAGA_BF16) return launch_saga_tc(p, mode, s.d, gp, st);
+  return launch_saga_split(p, mode, s.dtype, s.d, gp, st);
+}
+
 // Select + PV over the stored thresholds, then the combine.
 saga_status run_step(const saga_shape &s, const Plan &pl, StepParams p, int mode,
                      float *out, int32_t *sel_count, cudaStream_t st) {
-  cudaError_t e = launch_saga_split(p, mode, s.dtype, s.d, group_pad(s), st);
+  cudaError_t e = launch_split(s, p, mode, st);
   if (e != cudaSuccess) return SAGA_ERR_CUDA;
   e = launch_combine(p.partials, p.l_kv, p.err, out, sel_count, s.B, s.h_q, s.d, pl.S,
                      pl.split_len, s.cap, s.max_l_kv, st);
@@ -177,7 +186,7 @@ saga_status saga_refresh_threshold(const saga_shape *shape, const void *q, const
                     : reinterpret_cast<float *>(static_cast<char *>(ws) + pl.off_scores);
   // 1. score rows
   p.scores_out = rows;
-  cudaError_t e = launch_saga_split(p, kModeDump, s.dtype, s.d, group_pad(s), st);
+  cudaError_t e = launch_split(s, p, kModeDump, st);
   if (e != cudaSuccess) return SAGA_ERR_CUDA;
   // 2. exact N-th largest per row
   e = launch_radix_select(rows, s.max_l_kv, l_kv, p.err, N, tau, s.B, s.h_q, s.cap, s.max_l_kv,
@@ -227,8 +236,7 @@ saga_status saga_debug_scores(const saga_shape *shape, const void *q, const void
   StepParams p = base_params(s, pl, q, K, nullptr, l_kv, ws);
   p.partials = nullptr;
   p.scores_out = scores;
-  return cuda_status(launch_saga_split(p, kModeDump, s.dtype, s.d, group_pad(s),
-                                       reinterpret_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_split(s, p, kModeDump, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 saga_status saga_read_device_error(void *ws, saga_stream_t stream, int32_t *flags) {
