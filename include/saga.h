@@ -160,6 +160,38 @@ saga_status gqa_dense_decode(const saga_shape *shape, const void *q,
                              size_t ws_bytes, saga_stream_t stream);
 
 /*
+ * saga_decode_step without a workspace argument, for callers that cannot
+ * allocate device memory (for example code running inside an allocator's
+ * own callbacks, or a runtime that only hands out its preallocated pools and
+ * forbids cudaMalloc after start-up). It does exactly what saga_decode_step
+ * does with sel_mask = NULL, but keeps its scratch (error word and per-split
+ * softmax states) in one fixed array of SAGA_NOALLOC_SCRATCH_BYTES compiled
+ * into the library; every GPU that loads the library holds that array until
+ * the process exits. The paper has no counterpart to this entry point.
+ *   - The step needs 256 + 4*B*h_q*S*(d+4) bytes of scratch, S being the
+ *     number of l_kv splits the library plans (at most a few hundred); a
+ *     shape needing more than SAGA_NOALLOC_SCRATCH_BYTES is rejected with
+ *     SAGA_ERR_WORKSPACE, an invalid one with SAGA_ERR_INVALID_ARG, and
+ *     nothing is enqueued then. (The 16-layer batch-8 128K workload needs
+ *     2.6 MB per layer call.)
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine.
+ *   - The first call on each device looks up the array's device address
+ *     with that device current; make that first call before any stream
+ *     capture on the device.
+ *   - All calls on a device share the one array, which keeps the previous
+ *     call's contents: calls that can overlap on the GPU (different streams
+ *     without ordering) race on it and must be serialised by the caller.
+ *   - The device error word lives in that array and cannot be read back;
+ *     out-of-range lengths are still clamped exactly as in saga_decode_step.
+ */
+#define SAGA_NOALLOC_SCRATCH_BYTES (4u << 20)
+saga_status saga_decode_step_noalloc(const saga_shape *shape, const void *q,
+                                     const void *K, const void *V,
+                                     const int32_t *l_kv, const float *tau,
+                                     float *out, int32_t *sel_count,
+                                     saga_stream_t stream);
+
+/*
  * Write the fp32 score rows A[b][j][t], t < l_kv[b], into
  * scores [B][h_q][max_l_kv], with the same arithmetic as every other entry
  * point. For checking. Uses the workspace's error word only.

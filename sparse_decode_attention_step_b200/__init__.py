@@ -56,6 +56,7 @@ _SIGS = {
                                               _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "gqa_dense_decode": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "saga_debug_scores": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "saga_decode_step_noalloc": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P, _P, _P]),
     "saga_read_device_error": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_int32)]),
     "saga_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
@@ -159,6 +160,17 @@ def gqa_dense_decode(shp, q, K, V, l_kv, out, ws, stream=None):
     p, n = _ws(ws)
     _check(load().gqa_dense_decode(ctypes.byref(shp), _ptr(q), _ptr(K), _ptr(V), _ptr(l_kv),
                                    _ptr(out), p, n, _stream(stream)), "gqa_dense_decode")
+
+
+NOALLOC_SCRATCH_BYTES = 4 << 20
+
+
+def decode_step_noalloc(shp, q, K, V, l_kv, tau, out, sel_count=None, stream=None):
+    """saga_decode_step with the library's fixed device scratch instead of a
+    workspace, for callers that cannot allocate device memory."""
+    _check(load().saga_decode_step_noalloc(ctypes.byref(shp), _ptr(q), _ptr(K), _ptr(V),
+                                           _ptr(l_kv), _ptr(tau), _ptr(out), _ptr(sel_count),
+                                           _stream(stream)), "saga_decode_step_noalloc")
 
 
 def debug_scores(shp, q, K, l_kv, scores, ws, stream=None):

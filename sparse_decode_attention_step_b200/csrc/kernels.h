@@ -32,4 +32,11 @@ cudaError_t launch_radix_select(const float *scores, int64_t row_stride, const i
 // Dense GQA split kernel over grid (S, B * h_k), h_k == h_v; gp = h_q / h_k rounded up to 4.
 cudaError_t launch_dense_split(const StepParams &p, int dtype, int d, int gp, cudaStream_t st);
 
+// Plain step with a caller-chosen scratch buffer (see saga_decode_step_noalloc).
+size_t plain_step_scratch_bytes(const saga_shape &s);
+saga_status plain_step_with_scratch(const saga_shape *shape, const void *q, const void *K,
+                                    const void *V, const int32_t *l_kv, const float *tau,
+                                    float *out, int32_t *sel_count, void *scratch,
+                                    size_t scratch_bytes, cudaStream_t st);
+
 }  // namespace saga

@@ -116,6 +116,31 @@ saga_status run_step(const saga_shape &s, const Plan &pl, StepParams p, int mode
 }
 
 }  // namespace
+
+// Scratch a plain step needs (error word + per-split states; no score rows).
+size_t plain_step_scratch_bytes(const saga_shape &s) { return make_plan(s).off_scores; }
+
+// saga_decode_step's checks and launches with a caller-chosen scratch buffer
+// in place of the workspace (sel_mask not supported).
+saga_status plain_step_with_scratch(const saga_shape *shape, const void *q, const void *K,
+                                    const void *V, const int32_t *l_kv, const float *tau,
+                                    float *out, int32_t *sel_count, void *scratch,
+                                    size_t scratch_bytes, cudaStream_t st) {
+  saga_status r = check_shape(shape);
+  if (r != SAGA_OK) return r;
+  const saga_shape &s = *shape;
+  if ((r = check_inputs(s, q, K, l_kv)) != SAGA_OK) return r;
+  if (V == nullptr || !aligned(V, 16) || tau == nullptr || out == nullptr ||
+      !aligned(tau, 4) || !aligned(out, 16) || (sel_count && !aligned(sel_count, 4)))
+    return SAGA_ERR_INVALID_ARG;
+  if (scratch == nullptr || !aligned(scratch, kAlign) || scratch_bytes < plain_step_scratch_bytes(s))
+    return SAGA_ERR_WORKSPACE;
+  const Plan pl = make_plan(s);
+  StepParams p = base_params(s, pl, q, K, V, l_kv, scratch);
+  p.tau = tau;
+  return run_step(s, pl, p, kModeStep, out, sel_count, st);
+}
+
 }  // namespace saga
 
 using namespace saga;
