@@ -1,6 +1,6 @@
 // Thin wrappers over the sm_100a instructions the tensor-core score kernel
 // uses: mbarriers, TMA tile loads, tcgen05 MMA / TMEM, and their fences.
-// Every wait is bounded: it gives up after kWaitLimit polls and reports it.
+// Every wait is bounded: it gives up after kWaitLimitNs and reports it.
 #pragma once
 
 #include <cuda.h>
@@ -9,7 +9,8 @@
 namespace saga {
 namespace sm100 {
 
-constexpr uint32_t kWaitLimit = 1u << 20;   // polls before a wait gives up
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // a wait gives up after 2 s
+constexpr uint32_t kSuspendHintNs = 20000;          // sleep per poll while the phase is open
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -46,11 +47,36 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete; false on timeout.
+// try_wait that may suspend the thread until the phase completes or
+// `hint_ns` elapse, so a waiting warp does not take issue slots.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for the phase with the given parity to complete; false once
+// kWaitLimitNs have passed without it.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kWaitLimit; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
-  return false;
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, kSuspendHintNs)) return true;
+    if (global_ns() - t0 > kWaitLimitNs) return false;
+  }
 }
 
 // 4-D tiled TMA load (no multicast) into shared memory, completing on `bar`.
@@ -134,6 +160,11 @@ __device__ __forceinline__ uint64_t desc_k_sw128(uint32_t smem_addr) {
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Hint: bring the 128-byte line holding `p` into L2.
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
 __device__ __forceinline__ void named_bar(int id, int nthreads) {
