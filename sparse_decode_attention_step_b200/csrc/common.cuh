@@ -22,6 +22,8 @@ struct StepParams {
   float *scores_out;        // dump mode: [B][h_q][row_stride]
   float *partials;          // [B][h_q][S][d + kRecPad]
   uint8_t *sel_mask;        // nullable [B][h_q][row_stride]
+  uint32_t *hist;           // nullable [B][h_q][256]: dump mode adds the top-byte histogram
+                            // of each score row's order keys
   int32_t *err;             // device error word
   int64_t q_sb, q_sh, k_sb, k_sh, v_sb, v_sh;
   int64_t cap, max_l_kv, row_stride;

@@ -25,9 +25,11 @@ cudaError_t launch_combine(const float *partials, const int32_t *l_kv, int32_t *
                            cudaStream_t st);
 
 // tau[b][j] = N-th largest of the stored score row (b, j), or -inf if N >= l_kv[b].
+// hist0: nullable [B][h_q][256] top-byte histograms of the rows' order keys
+// (from the score pass); without it the kernel makes one more pass.
 cudaError_t launch_radix_select(const float *scores, int64_t row_stride, const int32_t *l_kv,
-                                int32_t *err, int N, float *tau, int B, int h_q, int64_t cap,
-                                int64_t max_l_kv, cudaStream_t st);
+                                int N, float *tau, int B, int h_q, int64_t cap, int64_t max_l_kv,
+                                const uint32_t *hist0, cudaStream_t st);
 
 // Dense GQA split kernel over grid (S, B * h_k), h_k == h_v; gp = h_q / h_k rounded up to 4.
 cudaError_t launch_dense_split(const StepParams &p, int dtype, int d, int gp, cudaStream_t st);

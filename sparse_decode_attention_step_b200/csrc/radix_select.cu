@@ -2,11 +2,19 @@
 // is reused between refreshes), by MSB-first radix selection over the
 // order-preserving uint32 keys of the fp32 scores.
 //
-// Pass p fixes bits [31-8p .. 24-8p] of the answer: a 256-bin histogram of
-// that digit over the elements whose higher bits equal the prefix fixed so
-// far, then a scan from the top bin down to the bin that holds the
-// remaining rank. After four passes the prefix is the full key of an
+// Digit p (p = 0..3) is bits [31-8p .. 24-8p] of the answer: a 256-bin
+// histogram of that digit over the elements whose higher bits equal the
+// prefix fixed so far, then a scan from the top bin down to the bin that holds
+// the remaining rank. After four digits the prefix is the full key of an
 // element of the row, so tau is always one of the row's own scores.
+//
+// One CTA per row. Digit 0 comes from the histogram the score pass already
+// built (or from one pass over the row). A second pass over the row fixes
+// digit 1 and copies the keys of the digit-0 bucket into shared memory; the
+// last two digits are found there. When that bucket does not fit (its scores
+// share one binade), a third pass copies only the keys that match the first
+// two digits; only if even those do not fit, digits 2 and 3 take one pass
+// over the row each.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -15,13 +23,91 @@ namespace saga {
 namespace {
 
 constexpr int kThreads = 1024;
+constexpr int kCand = 32768;                        // candidate keys kept on chip (128 KB)
 
-__global__ void __launch_bounds__(kThreads)
+struct Shared {
+  uint32_t hist[256];
+  uint32_t digit, rem, n_cand;
+};
+
+// Histogram of digit `shift` over keys with (k & mask) == prefix, one shared
+// atomic per distinct bin in a warp. All threads of the CTA call it.
+__device__ __forceinline__ void count_key(uint32_t k, bool valid, uint32_t mask, uint32_t prefix,
+                                          int shift, uint32_t *hist, int lane) {
+  const bool in = valid && (k & mask) == prefix;
+  const uint32_t active = __ballot_sync(0xffffffffu, in);
+  if (in) {
+    const uint32_t bin = (k >> shift) & 0xFFu;
+    const uint32_t peers = __match_any_sync(active, bin);
+    if (lane == __ffs(peers) - 1) atomicAdd(&hist[bin], static_cast<uint32_t>(__popc(peers)));
+  }
+}
+
+// Warp 0 finds the bin holding rank `rem` (1-based, counted from the top)
+// and stores it with the rank left inside that bin.
+__device__ __forceinline__ void pick_digit(Shared &sh, int lane) {
+  uint32_t c[8], sum = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) { c[e] = sh.hist[255 - 8 * lane - e]; sum += c[e]; }
+  uint32_t incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const uint32_t rem = sh.rem;
+  const uint32_t hit = __ballot_sync(0xffffffffu, incl >= rem);
+  const int owner = __ffs(hit) - 1;                 // rem <= bucket count, so hit != 0
+  if (lane == owner) {
+    uint32_t cum = incl - sum;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      if (cum + c[e] >= rem) {
+        sh.digit = 255 - 8 * lane - e;
+        sh.rem = rem - cum;
+        break;
+      }
+      cum += c[e];
+    }
+  }
+}
+
+// Visit every element t < L of a row as f(key, valid), all threads of the
+// CTA in step (f may use warp votes). Each thread keeps kVec * 4 elements in
+// flight per step (16-byte loads when the row is 16-byte aligned).
+constexpr int kVec = 4;
+template <typename F>
+__device__ __forceinline__ void for_row(const float *row, int64_t L, int tid, F f) {
+  constexpr int64_t kStep = static_cast<int64_t>(kThreads) * kVec * 4;
+  const bool vec = (reinterpret_cast<uintptr_t>(row) & 15u) == 0;
+  for (int64_t t0 = 0; t0 < L; t0 += kStep) {
+    float v[kVec][4];
+#pragma unroll
+    for (int u = 0; u < kVec; ++u) {
+      const int64_t i = t0 + (static_cast<int64_t>(u) * kThreads + tid) * 4;
+      if (vec && i + 3 < L) {
+        const float4 x = __ldg(reinterpret_cast<const float4 *>(row + i));
+        v[u][0] = x.x; v[u][1] = x.y; v[u][2] = x.z; v[u][3] = x.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[u][e] = i + e < L ? __ldg(row + i + e) : 0.f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kVec; ++u) {
+      const int64_t i = t0 + (static_cast<int64_t>(u) * kThreads + tid) * 4;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) f(order_key(v[u][e]), i + e < L);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
 radix_select_kernel(const float *__restrict__ scores, int64_t row_stride,
-                    const int32_t *__restrict__ l_kv, int32_t *err, int N,
-                    float *__restrict__ tau, int h_q, int64_t cap, int64_t max_l_kv) {
-  __shared__ uint32_t hist[256];
-  __shared__ uint32_t s_digit, s_rem;
+                    const int32_t *__restrict__ l_kv, int N, float *__restrict__ tau, int h_q,
+                    int64_t cap, int64_t max_l_kv, const uint32_t *__restrict__ hist0) {
+  __shared__ Shared sh;
+  extern __shared__ uint32_t cand[];
   const int bj = blockIdx.x;
   const int b = bj / h_q;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -34,59 +120,94 @@ radix_select_kernel(const float *__restrict__ scores, int64_t row_stride,
     return;
   }
   const float *row = scores + static_cast<int64_t>(bj) * row_stride;
-  uint32_t prefix = 0, mask = 0, rem = static_cast<uint32_t>(N);
+  if (tid == 0) { sh.rem = static_cast<uint32_t>(N); sh.n_cand = 0; }
 
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    for (int i = tid; i < 256; i += kThreads) hist[i] = 0;
+  // ---- digit 0: from the score pass's histogram, or one pass here ---------
+  if (hist0 != nullptr) {
+    for (int i = tid; i < 256; i += kThreads) sh.hist[i] = hist0[static_cast<int64_t>(bj) * 256 + i];
     __syncthreads();
-    for (int64_t t0 = 0; t0 < L; t0 += kThreads) {
-      const int64_t t = t0 + tid;
-      bool in = false;
-      uint32_t bin = 0;
-      if (t < L) {
-        const uint32_t k = order_key(row[t]);
-        in = (k & mask) == prefix;
-        bin = (k >> shift) & 0xFFu;
-      }
-      const uint32_t active = __ballot_sync(0xffffffffu, in);
+  } else {
+    for (int i = tid; i < 256; i += kThreads) sh.hist[i] = 0u;
+    __syncthreads();
+    for_row(row, L, tid, [&](uint32_t k, bool valid) {
+      count_key(k, valid, 0u, 0u, 24, sh.hist, lane);
+    });
+    __syncthreads();
+  }
+  if (warp == 0) pick_digit(sh, lane);
+  __syncthreads();
+  uint32_t prefix = sh.digit << 24, mask = 0xFF000000u;
+  __syncthreads();
+
+  // ---- digit 1: one pass over the row; keep the digit-0 bucket on chip -----
+  for (int i = tid; i < 256; i += kThreads) sh.hist[i] = 0u;
+  __syncthreads();
+  for_row(row, L, tid, [&](uint32_t k, bool valid) {
+    const bool in = valid && (k & mask) == prefix;
+    const uint32_t bal = __ballot_sync(0xffffffffu, in);
+    if (bal != 0u) {
+      uint32_t base = 0;
+      if (lane == 0) base = atomicAdd(&sh.n_cand, static_cast<uint32_t>(__popc(bal)));
+      base = __shfl_sync(0xffffffffu, base, 0);
       if (in) {
-        // one shared atomic per distinct bin in the warp
-        const uint32_t peers = __match_any_sync(active, bin);
-        if (lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+        const uint32_t at = base + __popc(bal & ((1u << lane) - 1u));
+        if (at < static_cast<uint32_t>(kCand)) cand[at] = k;
       }
     }
+    count_key(k, valid, mask, prefix, 16, sh.hist, lane);
+  });
+  __syncthreads();
+  if (warp == 0) pick_digit(sh, lane);
+  __syncthreads();
+  prefix |= sh.digit << 16;
+  mask |= 0x00FF0000u;
+  uint32_t n_cand = sh.n_cand;
+  bool on_chip = n_cand <= static_cast<uint32_t>(kCand);
+  __syncthreads();
+  if (!on_chip) {
+    // the top-byte bucket was too big: collect the (much smaller) bucket of
+    // the 16-bit prefix instead, with one more pass over the row
+    if (tid == 0) sh.n_cand = 0;
     __syncthreads();
-    if (warp == 0) {
-      // lane l owns bins 255-8l .. 248-8l (descending)
-      uint32_t c[8], sum = 0;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) { c[e] = hist[255 - 8 * lane - e]; sum += c[e]; }
-      uint32_t incl = sum;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      const uint32_t hit = __ballot_sync(0xffffffffu, incl >= rem);
-      const int owner = __ffs(hit) - 1;   // rem <= count of the prefix bucket, so hit != 0
-      if (lane == owner) {
-        uint32_t cum = incl - sum;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          if (cum + c[e] >= rem) {
-            s_digit = 255 - 8 * lane - e;
-            s_rem = rem - cum;
-            break;
-          }
-          cum += c[e];
+    for_row(row, L, tid, [&](uint32_t k, bool valid) {
+      const bool in = valid && (k & mask) == prefix;
+      const uint32_t bal = __ballot_sync(0xffffffffu, in);
+      if (bal != 0u) {
+        uint32_t base = 0;
+        if (lane == 0) base = atomicAdd(&sh.n_cand, static_cast<uint32_t>(__popc(bal)));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (in) {
+          const uint32_t at = base + __popc(bal & ((1u << lane) - 1u));
+          if (at < static_cast<uint32_t>(kCand)) cand[at] = k;
         }
       }
+    });
+    __syncthreads();
+    n_cand = sh.n_cand;
+    on_chip = n_cand <= static_cast<uint32_t>(kCand);
+    __syncthreads();
+  }
+
+  // ---- digits 2 and 3: over the candidates, else over the row -------------
+  for (int shift = 8; shift >= 0; shift -= 8) {
+    for (int i = tid; i < 256; i += kThreads) sh.hist[i] = 0u;
+    __syncthreads();
+    if (on_chip) {
+      for (uint32_t i0 = 0; i0 < n_cand; i0 += kThreads) {
+        const uint32_t i = i0 + tid;
+        const uint32_t k = i < n_cand ? cand[i] : 0u;
+        count_key(k, i < n_cand, mask, prefix, shift, sh.hist, lane);
+      }
+    } else {
+      for_row(row, L, tid, [&](uint32_t k, bool valid) {
+        count_key(k, valid, mask, prefix, shift, sh.hist, lane);
+      });
     }
     __syncthreads();
-    prefix |= s_digit << shift;
+    if (warp == 0) pick_digit(sh, lane);
+    __syncthreads();
+    prefix |= sh.digit << shift;
     mask |= 0xFFu << shift;
-    rem = s_rem;
     __syncthreads();
   }
   if (tid == 0) tau[bj] = from_order_key(prefix);
@@ -95,10 +216,18 @@ radix_select_kernel(const float *__restrict__ scores, int64_t row_stride,
 }  // namespace
 
 cudaError_t launch_radix_select(const float *scores, int64_t row_stride, const int32_t *l_kv,
-                                int32_t *err, int N, float *tau, int B, int h_q, int64_t cap,
-                                int64_t max_l_kv, cudaStream_t st) {
-  radix_select_kernel<<<B * h_q, kThreads, 0, st>>>(scores, row_stride, l_kv, err, N, tau, h_q,
-                                                   cap, max_l_kv);
+                                int N, float *tau, int B, int h_q, int64_t cap, int64_t max_l_kv,
+                                const uint32_t *hist0, cudaStream_t st) {
+  static bool attr_set = false;
+  const int smem = kCand * static_cast<int>(sizeof(uint32_t));
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(radix_select_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  radix_select_kernel<<<B * h_q, kThreads, smem, st>>>(scores, row_stride, l_kv, N, tau, h_q,
+                                                       cap, max_l_kv, hist0);
   return cudaGetLastError();
 }
 

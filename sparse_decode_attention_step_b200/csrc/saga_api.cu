@@ -22,7 +22,7 @@ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 struct Plan {
   int S;                    // splits per (b, key head)
   int64_t split_len;        // positions per split
-  size_t off_partials, off_scores, total;
+  size_t off_partials, off_scores, off_hist, total;
 };
 
 // Splits sized so the grid holds about kTargetCtas CTAs of equal length.
@@ -36,7 +36,8 @@ Plan make_plan(const saga_shape &s) {
   const size_t rec = static_cast<size_t>(s.d + kRecPad) * sizeof(float);
   p.off_partials = kAlign;   // [0, 256): device error word
   p.off_scores = align_up(p.off_partials + static_cast<size_t>(s.B) * s.h_q * p.S * rec);
-  p.total = align_up(p.off_scores + static_cast<size_t>(s.B) * s.h_q * s.max_l_kv * sizeof(float));
+  p.off_hist = align_up(p.off_scores + static_cast<size_t>(s.B) * s.h_q * s.max_l_kv * sizeof(float));
+  p.total = align_up(p.off_hist + static_cast<size_t>(s.B) * s.h_q * 256 * sizeof(uint32_t));
   return p;
 }
 
@@ -209,20 +210,32 @@ saga_status saga_refresh_threshold(const saga_shape *shape, const void *q, const
   float *rows = scores != nullptr
                     ? scores
                     : reinterpret_cast<float *>(static_cast<char *>(ws) + pl.off_scores);
-  // 1. score rows
+  // 1. score rows (bf16: with the top-byte histogram of every row)
+  uint32_t *hist = nullptr;
+  if (s.dtype == SAGA_BF16) {
+    hist = reinterpret_cast<uint32_t *>(static_cast<char *>(ws) + pl.off_hist);
+    if (cudaMemsetAsync(hist, 0, static_cast<size_t>(s.B) * s.h_q * 256 * sizeof(uint32_t), st) !=
+        cudaSuccess)
+      return SAGA_ERR_CUDA;
+  }
   p.scores_out = rows;
+  p.hist = hist;
   cudaError_t e = launch_split(s, p, kModeDump, st);
   if (e != cudaSuccess) return SAGA_ERR_CUDA;
   // 2. exact N-th largest per row
-  e = launch_radix_select(rows, s.max_l_kv, l_kv, p.err, N, tau, s.B, s.h_q, s.cap, s.max_l_kv,
+  e = launch_radix_select(rows, s.max_l_kv, l_kv, N, tau, s.B, s.h_q, s.cap, s.max_l_kv, hist,
                           st);
   if (e != cudaSuccess) return SAGA_ERR_CUDA;
   if (V == nullptr) return SAGA_OK;
-  // 3. this step's select + PV from the same rows, with the fresh tau
+  // 3. this step's select + PV with the fresh tau. bf16: the tensor-core step
+  // kernel recomputes the scores with the same MMAs, so they equal the rows
+  // tau came from bit for bit; fp32: the stored rows are read back.
   p.scores_out = nullptr;
-  p.scores_in = rows;
+  p.hist = nullptr;
   p.tau = tau;
   p.sel_mask = sel_mask;
+  if (s.dtype == SAGA_BF16) return run_step(s, pl, p, kModeStep, out, sel_count, st);
+  p.scores_in = rows;
   return run_step(s, pl, p, kModeFromScores, out, sel_count, st);
 }
 

@@ -166,6 +166,11 @@ saga_tc_kernel(const StepParams p, const int mode, const __grid_constant__ CUten
     }
     sm100::fence_proxy_async_smem();
     if (tid < kN) tau_s[tid] = (tid < G && mode != kModeDump) ? p.tau[b * p.h_q + j0 + tid] : 0.f;
+    if (mode == kModeDump && p.hist != nullptr) {
+      // the head lists are unused when dumping: they hold the score histograms
+      uint32_t *hs = reinterpret_cast<uint32_t *>(smem + Lo::off_key);
+      for (int i = tid; i < kN * 256; i += kThreads) hs[i] = 0u;
+    }
   }
   sm100::tc_fence_before();
   __syncthreads();
@@ -357,6 +362,21 @@ saga_tc_kernel(const StepParams p, const int mode, const __grid_constant__ CUten
         for (int g = 0; g < GP; ++g)
           if (g < G) p.scores_out[row0 + g * p.row_stride + t] = A[g];
       }
+      if (p.hist != nullptr) {
+        // top byte of each score's order key, one shared atomic per distinct
+        // bin in the warp
+        uint32_t(*hs)[256] = reinterpret_cast<uint32_t(*)[256]>(smem + Lo::off_key);
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+          const bool in = valid && g < G;
+          const uint32_t active = __ballot_sync(0xffffffffu, in);
+          if (in) {
+            const uint32_t bin = order_key(A[g]) >> 24;
+            const uint32_t peers = __match_any_sync(active, bin);
+            if (lane == __ffs(peers) - 1) atomicAdd(&hs[g][bin], static_cast<uint32_t>(__popc(peers)));
+          }
+        }
+      }
     } else {
       uint32_t selbits = 0;
 #pragma unroll
@@ -395,7 +415,17 @@ saga_tc_kernel(const StepParams p, const int mode, const __grid_constant__ CUten
     sm100::tc_fence_after();
     sm100::tmem_dealloc(tmem_base, kTmemCols);
   }
-  if (mode == kModeDump || bad || aborted(hdr)) return;
+  if (mode == kModeDump) {
+    if (p.hist != nullptr && !bad && !aborted(hdr)) {
+      const uint32_t *hs = reinterpret_cast<const uint32_t *>(smem + Lo::off_key);
+      for (int i = tid; i < G * 256; i += kComputeThreads) {
+        const uint32_t v = hs[i];
+        if (v != 0u) atomicAdd(&p.hist[static_cast<int64_t>(b * p.h_q + j0 + i / 256) * 256 + (i % 256)], v);
+      }
+    }
+    return;
+  }
+  if (bad || aborted(hdr)) return;
 
   // ---- merge the two halves of each head and write the split's record -----
   // (the K stages are idle now: every tile landed and was consumed)
