@@ -14,9 +14,13 @@ enum { kModeDump = 0, kModeStep = 1, kModeFromScores = 2 };
 cudaError_t launch_saga_split(const StepParams &p, int mode, int dtype, int d, int gp,
                               cudaStream_t st);
 
-// Tensor-core split kernel (bf16 caches, d in {64, 128}, h_q/h_k <= 16):
-// dump and step modes, bit-identical scores between the two.
-cudaError_t launch_saga_tc(const StepParams &p, int mode, int d, int gp, cudaStream_t st);
+// Persistent tensor-core split kernel: dump and step modes, bit-identical
+// scores between the two. Shapes it takes: saga_tc_supports.
+cudaError_t launch_saga_tc(const StepParams &p, int mode, int d, cudaStream_t st);
+
+// bf16 caches, d in {64, 128}, G = h_q / h_k <= 16, and the query heads of a
+// group fit four lane groups: (h_v / h_k) * ceil((h_q / h_v) / 4) <= 4.
+bool saga_tc_supports(int dtype, int d, int h_q, int h_k, int h_v);
 
 // Merge the per-split states of every (b, j) into out and sel_count.
 cudaError_t launch_combine(const float *partials, const int32_t *l_kv, int32_t *err,

@@ -12,8 +12,9 @@
 namespace saga {
 namespace {
 
-constexpr int64_t kTargetCtas = 4 * 148;   // four resident CTAs per B200 SM
-constexpr int64_t kSplitQuantum = 256;     // split lengths are multiples of a sub-chunk
+constexpr int64_t kSms = 148;              // B200 SMs: the persistent grid
+constexpr int64_t kTileKeys = 128;         // split lengths are multiples of a K tile
+constexpr int64_t kUnitTiles = 32;         // at most about this many tiles per split
 constexpr size_t kAlign = 256;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -25,13 +26,17 @@ struct Plan {
   size_t off_partials, off_scores, off_hist, total;
 };
 
-// Splits sized so the grid holds about kTargetCtas CTAs of equal length.
+// Splits of equal length (a multiple of the K tile) such that the
+// (b, kh, split) units number about a whole multiple of the SM count, with at
+// most about kUnitTiles tiles each.
 Plan make_plan(const saga_shape &s) {
   Plan p{};
-  const int64_t units = static_cast<int64_t>(s.B) * s.h_k;
-  const int64_t s_target = std::max<int64_t>(1, ceil_div(kTargetCtas, units));
+  const int64_t rows = static_cast<int64_t>(s.B) * s.h_k;
   const int64_t L = std::max<int64_t>(1, s.max_l_kv);
-  p.split_len = ceil_div(ceil_div(L, s_target), kSplitQuantum) * kSplitQuantum;
+  const int64_t tiles = rows * ceil_div(L, kTileKeys);
+  const int64_t waves = std::max<int64_t>(1, ceil_div(tiles, kSms * kUnitTiles));
+  const int64_t s_target = std::max<int64_t>(1, ceil_div(kSms * waves, rows));
+  p.split_len = ceil_div(ceil_div(L, s_target), kTileKeys) * kTileKeys;
   p.S = static_cast<int>(ceil_div(L, p.split_len));
   const size_t rec = static_cast<size_t>(s.d + kRecPad) * sizeof(float);
   p.off_partials = kAlign;   // [0, 256): device error word
@@ -97,13 +102,18 @@ int group_pad(const saga_shape &s) { return ((s.h_q / s.h_k) + 3) / 4 * 4; }
 
 saga_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SAGA_OK : SAGA_ERR_CUDA; }
 
-// Score-producing modes (dump, step) go to the tensor-core kernel for bf16
-// caches (a failure there is reported, never replaced by another path); fp32
-// caches and the from-scores mode use the SIMT split kernel.
+// The tensor-core kernel takes the score-producing modes (dump, step) of the
+// shapes it supports (a failure there is reported, never replaced by another
+// path); every other shape, and the from-scores mode, runs on the SIMT split
+// kernel. The choice depends on the shape alone, so a refresh and the steps
+// that follow it always see scores from the same kernel.
+bool use_tc(const saga_shape &s) {
+  return saga_tc_supports(s.dtype, s.d, s.h_q, s.h_k, s.h_v);
+}
+
 cudaError_t launch_split(const saga_shape &s, const StepParams &p, int mode, cudaStream_t st) {
-  const int gp = group_pad(s);
-  if (mode != kModeFromScores && s.dtype == SAGA_BF16) return launch_saga_tc(p, mode, s.d, gp, st);
-  return launch_saga_split(p, mode, s.dtype, s.d, gp, st);
+  if (mode != kModeFromScores && use_tc(s)) return launch_saga_tc(p, mode, s.d, st);
+  return launch_saga_split(p, mode, s.dtype, s.d, group_pad(s), st);
 }
 
 // Select + PV over the stored thresholds, then the combine.
@@ -210,9 +220,9 @@ saga_status saga_refresh_threshold(const saga_shape *shape, const void *q, const
   float *rows = scores != nullptr
                     ? scores
                     : reinterpret_cast<float *>(static_cast<char *>(ws) + pl.off_scores);
-  // 1. score rows (bf16: with the top-byte histogram of every row)
+  // 1. score rows (tensor-core kernel: with the top-byte histogram of every row)
   uint32_t *hist = nullptr;
-  if (s.dtype == SAGA_BF16) {
+  if (use_tc(s)) {
     hist = reinterpret_cast<uint32_t *>(static_cast<char *>(ws) + pl.off_hist);
     if (cudaMemsetAsync(hist, 0, static_cast<size_t>(s.B) * s.h_q * 256 * sizeof(uint32_t), st) !=
         cudaSuccess)
@@ -227,14 +237,14 @@ saga_status saga_refresh_threshold(const saga_shape *shape, const void *q, const
                           st);
   if (e != cudaSuccess) return SAGA_ERR_CUDA;
   if (V == nullptr) return SAGA_OK;
-  // 3. this step's select + PV with the fresh tau. bf16: the tensor-core step
-  // kernel recomputes the scores with the same MMAs, so they equal the rows
-  // tau came from bit for bit; fp32: the stored rows are read back.
+  // 3. this step's select + PV with the fresh tau. Tensor-core shapes: the
+  // step kernel recomputes the scores with the same MMAs, so they equal the
+  // rows tau came from bit for bit; other shapes read the stored rows back.
   p.scores_out = nullptr;
   p.hist = nullptr;
   p.tau = tau;
   p.sel_mask = sel_mask;
-  if (s.dtype == SAGA_BF16) return run_step(s, pl, p, kModeStep, out, sel_count, st);
+  if (use_tc(s)) return run_step(s, pl, p, kModeStep, out, sel_count, st);
   p.scores_in = rows;
   return run_step(s, pl, p, kModeFromScores, out, sel_count, st);
 }

@@ -1,31 +1,35 @@
 // Tensor-core split kernel for bf16 caches (sm_100a): Eq. 2 scores,
-// Atop-N item 1 compare and compaction, Eq. 7 sparse softmax + V gather, and
+// Atop-N item 1 compare, Eq. 7 sparse softmax with the V gather, and the
 // per-split online-softmax states, with the score contraction on tcgen05.
 //
-// One CTA per (sequence b, key head kh, split of l_kv): eight compute warps
-// and one TMA producer warp.
+// Persistent: one CTA per SM walks the work units (sequence b, key head kh,
+// split s of l_kv) u = blockIdx.x, blockIdx.x + gridDim.x, ... Warp roles:
 //
-//   producer    K tiles of 128 positions x d (bf16, 128B swizzle) stream by
-//               TMA into kStages shared-memory stages.
-//   scan phase  the compute warps walk the split in 256-position chunks.
-//               Thread 0 issues one chunk ahead the d/16 tcgen05.mma
-//               (M=128 keys, N=16 heads, K=16) per tile into a double-
-//               buffered TMEM accumulator; each thread then reads one key's
-//               16 head scores, scales them by 1/sqrt(d), compares them with
-//               tau and, for every head that keeps the key, appends (key,
-//               score) to its warp's list of that head (one ballot per head).
-//               The warps never hand tiles to one another; one barrier per
-//               chunk guards the TMEM reuse.
-//   gather      when the split is done (or a list is close to full) all
-//               eight warps turn to the V rows: 32 groups of 8 lanes, two per
-//               query head (one per half of the scan warps' lists), each lane
-//               gathering 16-byte chunks of 4 kept rows per round, with an
-//               online softmax per group. The two halves of each head merge
-//               at the end into the split's (m, l, acc) record.
-// Query heads beyond the group (G < 16) are zero rows of Q and never kept.
-// Every wait is bounded; on a timeout the CTA sets SAGA_DEVERR_TIMEOUT, lets
-// its copies and MMAs in flight land, frees TMEM and returns.
+//   warp 0      TMA producer: the unit's 16 query rows (one 16 x d tile) into
+//               a double-buffered Q operand, then the K tiles of 128
+//               positions x d (128B swizzle) through a ring of kStages
+//               stages. It runs ahead across unit boundaries.
+//   warp 1      MMA issuer and TMEM owner: per K tile d/16 tcgen05.mma
+//               (M = 128 keys, N = 16 query heads, K = 16) into one of kTBufs
+//               16-column TMEM buffers; the commits free the K stage and
+//               publish the scores.
+//   workers     4 x kRanks warps. Tile g belongs to rank g % kRanks; each of
+//               the four warps of that rank reads its TMEM lane quarter
+//               (32 keys x 16 heads), scales by 1/sqrt(d), compares with tau
+//               and then gathers V for its own kept keys: lane group v (8
+//               lanes) owns up to four query heads that share one value
+//               head, so each kept V row is read once for all of them, and
+//               keeps their online-softmax states in registers. At the end of
+//               a unit the workers' states merge in a shared-memory tree and
+//               worker 0 writes the unit's (m, l, count, acc) records.
+//
+// Query heads beyond the group (G < 16) are rows of other heads or zero rows
+// of Q; their tau is +inf, so they are never kept, and they are never dumped.
+// Every wait is bounded; on a timeout the CTA sets SAGA_DEVERR_TIMEOUT and
+// all roles stop, after the copies and MMAs in flight have landed.
 #include <cuda.h>
+
+#include <atomic>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -35,51 +39,135 @@ namespace saga {
 
 namespace {
 
-constexpr int kWarps = 8;                                  // compute warps
-constexpr int kComputeThreads = kWarps * 32;
-constexpr int kProducerWarp = kWarps;
-constexpr int kThreads = kComputeThreads + 32;             // 288
 constexpr int kTileKeys = 128;
-constexpr int kChunkKeys = 2 * kTileKeys;
-constexpr int kN = 16;                                     // MMA N: query heads, padded
-constexpr int kTmemCols = 64;                              // 2 chunks x 2 tiles x 16 heads
-constexpr int kBar = 1;                                    // named barrier of the compute warps
-constexpr int kUnroll = 4;                                 // kept rows in flight per lane group
+constexpr int kN = 16;                      // MMA N: query heads of a group, padded
+constexpr int kRows = 4;                    // kept V rows in flight per lane group
+constexpr int kWorkerBar = 1;               // named barrier of the worker warps
 constexpr uint32_t kIdesc = sm100::idesc_bf16_f32(kTileKeys, kN);
 constexpr float kLog2e = 1.4426950408889634f;
 
+constexpr int cmax(int a, int b) { return a > b ? a : b; }
+
 template <int D>
 struct Cfg {
-  static constexpr int kStages = D == 64 ? 3 : 2;
-  static constexpr int kBoxes = D / 64;                     // 64-column TMA boxes per tile
-  static constexpr int kBoxBytes = kTileKeys * 128;         // 128 rows x 128 bytes
+  static constexpr int kRanks = D == 64 ? 3 : 2;              // worker warps per lane quarter
+  static constexpr int kWorkers = 4 * kRanks;
+  static constexpr int kThreads = 32 * (2 + kWorkers);
+  static constexpr int kStages = D == 64 ? 8 : 4;             // 128 KB of K in flight
+  static constexpr int kTBufs = 2 * kRanks;                    // TMEM score buffers
+  static constexpr int kTmemCols = kTBufs * kN <= 32 ? 32 : (kTBufs * kN <= 64 ? 64 : 128);
+  static constexpr int kBoxes = D / 64;                        // 64-column TMA boxes per tile
+  static constexpr int kBoxBytes = kTileKeys * 128;
   static constexpr int kTileBytes = kBoxes * kBoxBytes;
-  static constexpr int kQBlockBytes = kN * 128;             // 16 rows x 128 bytes per box
-  static constexpr int kQBytes = kBoxes * kQBlockBytes;
-  static constexpr int kCap = D == 64 ? 48 : 40;           // kept keys per (head, warp) list
+  static constexpr int kQBoxBytes = kN * 128;
+  static constexpr int kQBytes = kBoxes * kQBoxBytes;
+  static constexpr int CPL = D / 64;                           // 16-byte chunks per lane per V row
+  static constexpr int EPL = 8 * CPL;                          // V row elements per lane
+  static constexpr int kRec = D + kRecPad;
+  static constexpr int kStateFloats = kN * kRec;               // one warp's 16 head states
+  static constexpr int kScoreBytes = kWorkers * 2 * 32 * kN * 4;   // two kept-score row sets per warp
+  static constexpr int kMergeBytes = kWorkers * (kStateFloats + kN) * 4;  // states + weights
+  static constexpr int kHistBytes = kN * 256 * 4;
+  static constexpr int kScratchBytes = cmax(cmax(kScoreBytes, kMergeBytes), kHistBytes);
 };
 
+template <int D>
 struct Header {
-  uint64_t full[4], empty[4];
-  uint64_t mma_done[2];
+  uint64_t full[Cfg<D>::kStages], empty[Cfg<D>::kStages];
+  uint64_t tfull[Cfg<D>::kTBufs], tempty[Cfg<D>::kTBufs];
+  uint64_t qfull[2], qempty[2];
   uint32_t tmem_base;
   int abort;
+  alignas(16) float tau[kN];
 };
 
 template <int D>
 struct Layout {
+  using C = Cfg<D>;
   static constexpr int off_stage = 0;
-  static constexpr int off_q = Cfg<D>::kStages * Cfg<D>::kTileBytes;
-  static constexpr int off_key = off_q + Cfg<D>::kQBytes;                // int [kN][kWarps][kCap]
-  static constexpr int off_sc = off_key + kN * kWarps * Cfg<D>::kCap * 4; // float, same shape
-  static constexpr int off_cnt = off_sc + kN * kWarps * Cfg<D>::kCap * 4; // int [kN][kWarps]
-  static constexpr int off_tau = off_cnt + kN * kWarps * 4;
-  static constexpr int off_hdr = off_tau + kN * 4;
-  static constexpr int bytes = off_hdr + static_cast<int>(sizeof(Header));
-  static constexpr int alloc = bytes + 1024;               // slack for 1024-byte alignment
+  static constexpr int off_q = C::kStages * C::kTileBytes;
+  static constexpr int off_scratch = off_q + 2 * C::kQBytes;
+  static constexpr int off_hdr = off_scratch + C::kScratchBytes;
+  static constexpr int bytes = off_hdr + static_cast<int>(sizeof(Header<D>));
+  static constexpr int alloc = bytes + 1024;                  // slack for 1024-byte alignment
+  static_assert(alloc <= 227 * 1024, "shared memory of one CTA");
+  static_assert(off_hdr % 16 == 0 && off_q % 1024 == 0, "operand alignment");
 };
 
-__device__ __forceinline__ bool bar_any(bool pred) {
+// Lane group v of a worker warp owns query heads hbase[v] .. hbase[v] + nh[v] - 1
+// of the group, all reading value head kh * (h_v / h_k) + vs[v]; smask[v] is
+// the same set as a 16-bit mask.
+struct HeadMap {
+  int hbase[4], nh[4], vs[4];
+  uint32_t smask[4];
+};
+
+// a[v] for a lane-dependent v without indexing the parameter array
+__device__ __forceinline__ int pick4(const int (&a)[4], int v) {
+  return v == 0 ? a[0] : (v == 1 ? a[1] : (v == 2 ? a[2] : a[3]));
+}
+
+struct Unit {
+  int b, kh, s;
+  int64_t t_begin, t_end;
+  int n_tiles;
+};
+
+// Work unit u; false when its split lies beyond l_kv[b] (nothing to do).
+__device__ __forceinline__ bool unit_at(const StepParams &p, int u, bool report, Unit &un) {
+  const int bk = u % (p.B * p.h_k);
+  un.s = u / (p.B * p.h_k);
+  un.b = bk / p.h_k;
+  un.kh = bk % p.h_k;
+  int64_t L;
+  if (report) {
+    L = clamp_len(p, un.b);
+  } else {
+    L = p.l_kv[un.b];
+    const int64_t hi = p.cap < p.max_l_kv ? p.cap : p.max_l_kv;
+    L = L < 0 ? 0 : (L > hi ? hi : L);
+  }
+  un.t_begin = static_cast<int64_t>(un.s) * p.split_len;
+  if (un.t_begin >= L) return false;
+  un.t_end = min(un.t_begin + p.split_len, L);
+  un.n_tiles = static_cast<int>((un.t_end - un.t_begin + kTileKeys - 1) / kTileKeys);
+  return true;
+}
+
+template <int D>
+__device__ __forceinline__ bool aborted(Header<D> *h) {
+  return *reinterpret_cast<volatile int *>(&h->abort) != 0;
+}
+
+template <int D>
+__device__ __forceinline__ void fail(const StepParams &p, Header<D> *h) {
+  if (!aborted(h)) atomicOr(p.err, SAGA_DEVERR_TIMEOUT);
+  *reinterpret_cast<volatile int *>(&h->abort) = 1;
+}
+
+// Bounded wait that also gives up as soon as another role has aborted.
+template <int D>
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Header<D> *h) {
+  if (sm100::mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = sm100::global_ns();
+  for (;;) {
+    if (sm100::mbar_try_wait_sleep(bar, parity, sm100::kSuspendHintNs)) return true;
+    if (aborted(h)) return false;
+    if (sm100::global_ns() - t0 > sm100::kWaitLimitNs) return false;
+  }
+}
+
+// Warp-uniform version: lane 0 waits, the verdict is broadcast.
+template <int D>
+__device__ __forceinline__ bool warp_wait_bar(uint64_t *bar, uint32_t parity, Header<D> *h) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, h);
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
+// OR of `pred` over the worker warps (a barrier among them).
+template <int D>
+__device__ __forceinline__ bool workers_any(bool pred) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
@@ -87,379 +175,430 @@ __device__ __forceinline__ bool bar_any(bool pred) {
       "bar.red.or.pred p, %2, %3, q;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(r)
-      : "r"(static_cast<uint32_t>(pred)), "r"(kBar), "r"(kComputeThreads)
+      : "r"(static_cast<uint32_t>(pred)), "r"(kWorkerBar), "r"(Cfg<D>::kWorkers * 32)
       : "memory");
   return r != 0;
 }
 
-__device__ __forceinline__ void fail(const StepParams &p, Header *h) {
-  atomicOr(p.err, SAGA_DEVERR_TIMEOUT);
-  *reinterpret_cast<volatile int *>(&h->abort) = 1;
+template <int D>
+__device__ __forceinline__ void workers_sync() {
+  sm100::named_bar(kWorkerBar, Cfg<D>::kWorkers * 32);
 }
 
-__device__ __forceinline__ bool aborted(Header *h) {
-  return *reinterpret_cast<volatile int *>(&h->abort) != 0;
+// Kept-score row of key k in a worker's scratch: 16 floats, 16-byte quads
+// rotated by the key so the four row stores of a warp spread over the banks.
+__device__ __forceinline__ int score_slot(int k, int h) {
+  return k * kN + ((((h >> 2) ^ (k >> 1)) & 3) << 2) + (h & 3);
 }
 
-// Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast.
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity) {
-  bool ok = true;
-  if ((threadIdx.x & 31) == 0) ok = sm100::mbar_wait(bar, parity);
-  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+// One worker state (m, l, count, acc over its lane's slice) into a record
+// laid out as {m, l, count, pad, acc[D]}; lane c8 == 0 writes the scalars.
+template <int EPL>
+__device__ __forceinline__ void put_state(float *r, int c8, float m, float l, int cnt,
+                                          const float (&acc)[EPL]) {
+  if (c8 == 0) {
+    r[0] = m;
+    r[1] = l;
+    r[2] = __int_as_float(cnt);
+    r[3] = 0.f;
+  }
+#pragma unroll
+  for (int cc = 0; cc < EPL / 8; ++cc) {
+    float4 *dst = reinterpret_cast<float4 *>(r + kRecPad + (c8 + 8 * cc) * 8);
+    dst[0] = make_float4(acc[8 * cc], acc[8 * cc + 1], acc[8 * cc + 2], acc[8 * cc + 3]);
+    dst[1] = make_float4(acc[8 * cc + 4], acc[8 * cc + 5], acc[8 * cc + 6], acc[8 * cc + 7]);
+  }
 }
 
-template <int D, int GP>
-__global__ void __launch_bounds__(kThreads, 2)
-saga_tc_kernel(const StepParams p, const int mode, const __grid_constant__ CUtensorMap kmap) {
+template <int D, int MODE>
+__global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
+saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
+               const __grid_constant__ CUtensorMap qmap, const HeadMap hm) {
   using C = Cfg<D>;
   using Lo = Layout<D>;
-  constexpr int CPL = D / 64;                // 16-byte chunks of a V row per gather lane
-  constexpr int EPL = 8 * CPL;               // row elements per gather lane
+  constexpr int CPL = C::CPL, EPL = C::EPL;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = sm100::smem_u32(smem_raw);
   uint8_t *smem = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
   uint8_t *stages = smem + Lo::off_stage;
-  uint16_t *qop = reinterpret_cast<uint16_t *>(smem + Lo::off_q);
-  int(*lkey)[kWarps][C::kCap] = reinterpret_cast<int(*)[kWarps][C::kCap]>(smem + Lo::off_key);
-  float(*lsc)[kWarps][C::kCap] = reinterpret_cast<float(*)[kWarps][C::kCap]>(smem + Lo::off_sc);
-  int(*lcnt)[kWarps] = reinterpret_cast<int(*)[kWarps]>(smem + Lo::off_cnt);
-  float *tau_s = reinterpret_cast<float *>(smem + Lo::off_tau);
-  Header *hdr = reinterpret_cast<Header *>(smem + Lo::off_hdr);
+  uint8_t *qbuf = smem + Lo::off_q;
+  float *scratch = reinterpret_cast<float *>(smem + Lo::off_scratch);
+  Header<D> *h = reinterpret_cast<Header<D> *>(smem + Lo::off_hdr);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int s = blockIdx.x;
-  const int b = blockIdx.y / p.h_k, kh = blockIdx.y % p.h_k;
   const int G = p.h_q / p.h_k;
-  const int j0 = kh * G;
-  const int64_t L = clamp_len(p, b);
-  const int64_t t_begin = static_cast<int64_t>(s) * p.split_len;
-  if (t_begin >= L) return;                      // uniform, before any barrier or TMEM
-  const int64_t t_end = min(t_begin + p.split_len, L);
-  const int n_tiles = static_cast<int>((t_end - t_begin + kTileKeys - 1) / kTileKeys);
-  const int n_chunks = (n_tiles + 1) / 2;
+  const int vpg = p.h_v / p.h_k;
+  const int n_units = p.B * p.h_k * p.S;
 
   // ---- set-up --------------------------------------------------------------
   if (tid == 0) {
     for (int i = 0; i < C::kStages; ++i) {
-      sm100::mbar_init(&hdr->full[i], 1);
-      sm100::mbar_init(&hdr->empty[i], 1);
+      sm100::mbar_init(&h->full[i], 1);
+      sm100::mbar_init(&h->empty[i], 1);
     }
-    sm100::mbar_init(&hdr->mma_done[0], 1);
-    sm100::mbar_init(&hdr->mma_done[1], 1);
-    hdr->abort = 0;
+    for (int i = 0; i < C::kTBufs; ++i) {
+      sm100::mbar_init(&h->tfull[i], 1);
+      sm100::mbar_init(&h->tempty[i], 4);     // the four lane-quarter warps of the rank
+    }
+    for (int i = 0; i < 2; ++i) {
+      sm100::mbar_init(&h->qfull[i], 1);
+      sm100::mbar_init(&h->qempty[i], 1);
+    }
+    h->abort = 0;
     sm100::fence_mbar_init();
   }
-  if (warp == 0) {
-    sm100::tmem_alloc(&hdr->tmem_base, kTmemCols);
+  if (warp == 1) {
+    sm100::tmem_alloc(&h->tmem_base, C::kTmemCols);
     sm100::tmem_relinquish();
   }
-  {
-    const uint16_t *qg = static_cast<const uint16_t *>(p.q) + b * p.q_sb;
-    for (int idx = tid; idx < kN * D; idx += kThreads) {
-      const int n = idx / D, k = idx % D;
-      const uint16_t v = n < G ? qg[(j0 + n) * p.q_sh + k] : static_cast<uint16_t>(0);
-      const int box = k / 64, kk = k % 64;
-      const int off = box * C::kQBlockBytes + (n / 8) * 1024 + (n % 8) * 128 +
-                      ((((kk * 2) >> 4) ^ (n % 8)) << 4) + ((kk * 2) & 15);
-      qop[off / 2] = v;
-    }
-    sm100::fence_proxy_async_smem();
-    if (tid < kN) tau_s[tid] = (tid < G && mode != kModeDump) ? p.tau[b * p.h_q + j0 + tid] : 0.f;
-    if (mode == kModeDump && p.hist != nullptr) {
-      // the head lists are unused when dumping: they hold the score histograms
-      uint32_t *hs = reinterpret_cast<uint32_t *>(smem + Lo::off_key);
-      for (int i = tid; i < kN * 256; i += kThreads) hs[i] = 0u;
-    }
+  if (MODE == kModeDump && p.hist != nullptr && warp >= 2) {
+    uint32_t *hs = reinterpret_cast<uint32_t *>(scratch);
+    for (int i = tid - 64; i < kN * 256; i += C::kWorkers * 32) hs[i] = 0u;
   }
   sm100::tc_fence_before();
   __syncthreads();
   sm100::tc_fence_after();
-  const uint32_t tmem_base = hdr->tmem_base;
+  const uint32_t tmem_base = h->tmem_base;
 
-  // ---- TMA producer ---------------------------------------------------------
-  if (warp == kProducerWarp) {
+  if (warp == 0) {
+    // ---- TMA producer ------------------------------------------------------
     if (lane == 0) {
       sm100::prefetch_tensormap(&kmap);
-      int issued = 0;
-      for (int i = 0; i < n_tiles; ++i) {
-        const int st = i % C::kStages, round = i / C::kStages;
-        if (aborted(hdr)) break;
-        if (!sm100::mbar_wait(&hdr->empty[st], (round & 1) ^ 1)) { fail(p, hdr); break; }
-        sm100::mbar_arrive_expect_tx(&hdr->full[st], C::kTileBytes);
-        const int y = static_cast<int>(t_begin) + i * kTileKeys;
+      sm100::prefetch_tensormap(&qmap);
+      uint32_t g = 0;
+      int k = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        Unit un;
+        if (!unit_at(p, u, true, un)) continue;
+        const int qb = k & 1;
+        if (!wait_bar(&h->qempty[qb], ((k >> 1) & 1) ^ 1, h)) { ok = false; break; }
+        sm100::mbar_arrive_expect_tx(&h->qfull[qb], C::kQBytes);
 #pragma unroll
         for (int bx = 0; bx < C::kBoxes; ++bx)
-          sm100::tma_load_4d(stages + st * C::kTileBytes + bx * C::kBoxBytes, &kmap,
-                             &hdr->full[st], bx * 64, y, kh, b);
-        issued = i + 1;
+          sm100::tma_load_3d(qbuf + qb * C::kQBytes + bx * C::kQBoxBytes, &qmap, &h->qfull[qb],
+                             bx * 64, un.kh * G, un.b);
+        ++k;
+        for (int i = 0; i < un.n_tiles; ++i) {
+          const int st = g % C::kStages;
+          if (!wait_bar(&h->empty[st], ((g / C::kStages) & 1) ^ 1, h)) { ok = false; break; }
+          sm100::mbar_arrive_expect_tx(&h->full[st], C::kTileBytes);
+          const int y = static_cast<int>(un.t_begin) + i * kTileKeys;
+#pragma unroll
+          for (int bx = 0; bx < C::kBoxes; ++bx)
+            sm100::tma_load_4d(stages + st * C::kTileBytes + bx * C::kBoxBytes, &kmap,
+                               &h->full[st], bx * 64, y, un.kh, un.b);
+          ++g;
+        }
       }
-      // every copy still in flight lands before the CTA can exit
-      for (int i = issued > C::kStages ? issued - C::kStages : 0; i < issued; ++i)
-        sm100::mbar_wait(&hdr->full[i % C::kStages], (i / C::kStages) & 1);
-    }
-    return;
-  }
-
-  // ---- compute warps --------------------------------------------------------
-  const uint32_t q_u32 = sm100::smem_u32(qop);
-  const uint32_t st_u32 = sm100::smem_u32(stages);
-  // Thread 0: the MMAs of chunk c (its one or two tiles) into TMEM set c & 1.
-  auto issue_chunk = [&](int c) -> bool {
-    for (int u = 0; u < 2 && 2 * c + u < n_tiles; ++u) {
-      const int tt = 2 * c + u;
-      const int st = tt % C::kStages;
-      if (!sm100::mbar_wait(&hdr->full[st], (tt / C::kStages) & 1)) return false;
-      sm100::tc_fence_after();
-      const uint32_t a0 = st_u32 + st * C::kTileBytes;
-#pragma unroll
-      for (int j = 0; j < D / 16; ++j) {
-        const int bx = j / 4, kk = j % 4;
-        const uint64_t ad = sm100::desc_k_sw128(a0 + bx * C::kBoxBytes + kk * 32);
-        const uint64_t bd = sm100::desc_k_sw128(q_u32 + bx * C::kQBlockBytes + kk * 32);
-        sm100::mma_bf16(tmem_base + (c & 1) * 2 * kN + u * kN, ad, bd, kIdesc, j > 0 ? 1u : 0u);
+      if (!ok) {
+        fail(p, h);
+        // the copies still in flight land before the CTA can exit: the
+        // last kStages K tiles and the last two Q tiles
+        for (uint32_t i = g > static_cast<uint32_t>(C::kStages) ? g - C::kStages : 0; i < g; ++i)
+          sm100::mbar_wait(&h->full[i % C::kStages], (i / C::kStages) & 1);
+        for (int i = k > 2 ? k - 2 : 0; i < k; ++i)
+          sm100::mbar_wait(&h->qfull[i & 1], (i >> 1) & 1);
       }
-      sm100::mma_commit(&hdr->empty[st]);
     }
-    sm100::mma_commit(&hdr->mma_done[c & 1]);
-    return true;
-  };
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---- MMA issuer ----------------------------------------------------------
+    if (lane == 0) {
+      const uint32_t st_u32 = sm100::smem_u32(stages);
+      const uint32_t q_u32 = sm100::smem_u32(qbuf);
+      uint32_t g = 0, committed = 0;
+      int k = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        Unit un;
+        if (!unit_at(p, u, false, un)) continue;
+        const int qb = k & 1;
+        if (!wait_bar(&h->qfull[qb], (k >> 1) & 1, h)) { ok = false; break; }
+        for (int i = 0; i < un.n_tiles; ++i) {
+          const int st = g % C::kStages, tb = g % C::kTBufs;
+          if (!wait_bar(&h->full[st], (g / C::kStages) & 1, h) ||
+              !wait_bar(&h->tempty[tb], ((g / C::kTBufs) & 1) ^ 1, h)) {
+            ok = false;
+            break;
+          }
+          sm100::tc_fence_after();
+          const uint32_t a0 = st_u32 + st * C::kTileBytes;
+          const uint32_t b0 = q_u32 + qb * C::kQBytes;
+#pragma unroll
+          for (int j = 0; j < D / 16; ++j) {
+            const int bx = j / 4, kk = j % 4;
+            const uint64_t ad = sm100::desc_k_sw128(a0 + bx * C::kBoxBytes + kk * 32);
+            const uint64_t bd = sm100::desc_k_sw128(b0 + bx * C::kQBoxBytes + kk * 32);
+            sm100::mma_bf16(tmem_base + tb * kN, ad, bd, kIdesc, j > 0 ? 1u : 0u);
+          }
+          sm100::mma_commit(&h->empty[st]);
+          sm100::mma_commit(&h->tfull[tb]);
+          ++g;
+          committed = g;
+        }
+        if (!ok) break;
+        sm100::mma_commit(&h->qempty[qb]);
+        ++k;
+      }
+      if (!ok) {
+        fail(p, h);
+        // every MMA issued has landed before TMEM and the stages go away
+        if (committed > 0)
+          sm100::mbar_wait(&h->tfull[(committed - 1) % C::kTBufs],
+                           ((committed - 1) / C::kTBufs) & 1);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---- workers ------------------------------------------------------------
+    const int widx = warp - 2;
+    const int quarter = warp & 3;             // TMEM lanes this warp may read
+    const int rank = widx >> 2;
+    const int v = lane >> 3, c8 = lane & 7;
+    const int hbase = pick4(hm.hbase, v), nh = pick4(hm.nh, v), vsl = pick4(hm.vs, v);
+    // two kept-score row sets, used in turn
+    float *rows_base = scratch + widx * 2 * 32 * kN;
+    uint32_t g = 0;
+    bool bad = false;
 
-  const int64_t row0 = static_cast<int64_t>(b * p.h_q + j0) * p.row_stride;
-  const uint32_t lt_mask = (1u << lane) - 1u;
-  int my_cnt = 0;                      // lane g < 16: this warp's kept keys of head g
-  // gather role: lane group (part, head)
-  const int unit = warp * 4 + (lane >> 3);
-  const int gh = unit % kN, part = unit / kN, c8 = lane & 7;
-  const bool live = gh < G && mode != kModeDump;
-  const int vh = live ? ((j0 + gh) * p.h_v) / p.h_q : 0;
-  const uint16_t *vrow = static_cast<const uint16_t *>(p.V) + b * p.v_sb + vh * p.v_sh;
-  float m_run = -INFINITY, l_run = 0.f, acc[EPL];
-  int cnt_run = 0;
-#pragma unroll
-  for (int v = 0; v < EPL; ++v) acc[v] = 0.f;
+    float m[4], l[4], acc[4][EPL];
+    int cnt[4];
+    const uint16_t *vrow = nullptr;
 
-  // All compute warps: fold the kept keys of every list into the lane
-  // groups' softmax states, then empty the lists.
-  auto gather = [&]() {
-    if (lane < kN) lcnt[lane][warp] = my_cnt;
-    sm100::named_bar(kBar, kComputeThreads);
-    int q1 = 0, q2 = 0, q3 = 0, ntot = 0;
-    if (live) {
-      const int w0 = 4 * part;
-      q1 = lcnt[gh][w0];
-      q2 = q1 + lcnt[gh][w0 + 1];
-      q3 = q2 + lcnt[gh][w0 + 2];
-      ntot = q3 + lcnt[gh][w0 + 3];
-    }
-    // entry e -> (list of scan warp w, slot)
-    auto locate = [&](int e, int &w, int &slot) {
-      const int k = (e >= q1) + (e >= q2) + (e >= q3);
-      const int base = k == 0 ? 0 : (k == 1 ? q1 : (k == 2 ? q2 : q3));
-      w = 4 * part + k;
-      slot = e - base;
-    };
-    const int gq = live ? gh : 0;
-    float mc = -INFINITY;
-    for (int e = c8; e < ntot; e += 8) {
-      int w, slot;
-      locate(e, w, slot);
-      mc = fmaxf(mc, lsc[gq][w][slot]);
-    }
+    // Fold the kept keys `mine` of this lane group (keys t0 + bit) into the
+    // lane group's online-softmax states, kRows V rows in flight per round.
+    auto gather = [&](uint32_t mine, int64_t t0, int64_t t_any, const float *rows) {
+      const int nmax = static_cast<int>(__reduce_max_sync(0xffffffffu, __popc(mine)));
+      for (int r0 = 0; r0 < nmax; r0 += kRows) {
+        uint4 raw[kRows][CPL];
+        float sc[kRows][4];
 #pragma unroll
-    for (int off = 1; off < 8; off <<= 1) mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, off));
-    const float m_new = fmaxf(m_run, mc);
-    const float corr = m_new == -INFINITY ? 1.f : exp2f((m_run - m_new) * kLog2e);
-    l_run *= corr;
+        for (int r = 0; r < kRows; ++r) {
+          const int kk = mine != 0u ? __ffs(mine) - 1 : -1;
+          mine &= mine - 1u;
+          // idle slots re-read a row of the unit, which always exists
+          const int64_t tr = kk >= 0 ? t0 + kk : t_any;
 #pragma unroll
-    for (int v = 0; v < EPL; ++v) acc[v] *= corr;
-    m_run = m_new;
-    int nmax = ntot;
+          for (int cc = 0; cc < CPL; ++cc)
+            raw[r][cc] = __ldg(reinterpret_cast<const uint4 *>(vrow + tr * D) + c8 + 8 * cc);
+          const int ks = kk >= 0 ? kk : 0;
 #pragma unroll
-    for (int off = 8; off < 32; off <<= 1) nmax = max(nmax, __shfl_xor_sync(0xffffffffu, nmax, off));
-    for (int e0 = 0; e0 < nmax; e0 += kUnroll) {
-      uint4 raw[kUnroll][CPL];
-      float sc[kUnroll];
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int e = e0 + u;
-        int64_t t = t_begin;                       // idle slots re-read a valid row
-        sc[u] = -INFINITY;
-        if (e < ntot) {
-          int w, slot;
-          locate(e, w, slot);
-          sc[u] = lsc[gq][w][slot];
-          t = t_begin + lkey[gq][w][slot];
+          for (int a = 0; a < 4; ++a) {
+            const int hd = min(hbase + a, kN - 1);
+            sc[r][a] = (kk >= 0 && a < nh) ? rows[score_slot(ks, hd)] : -INFINITY;
+          }
         }
 #pragma unroll
-        for (int cc = 0; cc < CPL; ++cc)
-          raw[u][cc] = __ldg(reinterpret_cast<const uint4 *>(vrow + t * D) + c8 + 8 * cc);
-      }
+        for (int a = 0; a < 4; ++a) {
+          float mx = sc[0][a];
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        if (e0 + u < ntot) {
-          const float pw = exp2f((sc[u] - m_run) * kLog2e);
-          l_run += pw;
-          cnt_run += 1;
+          for (int r = 1; r < kRows; ++r) mx = fmaxf(mx, sc[r][a]);
+          const float mn = fmaxf(m[a], mx);
+          const float corr = mn == m[a] ? 1.f : exp2f((m[a] - mn) * kLog2e);
+          m[a] = mn;
+          l[a] *= corr;
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) acc[a][e] *= corr;
+        }
+#pragma unroll
+        for (int r = 0; r < kRows; ++r) {
+          float vf[EPL];
 #pragma unroll
           for (int cc = 0; cc < CPL; ++cc) {
-            const uint4 x = raw[u][cc];
-            float *a8 = acc + 8 * cc;
-            a8[0] = fmaf(pw, bf16lo(x.x), a8[0]);
-            a8[1] = fmaf(pw, bf16hi(x.x), a8[1]);
-            a8[2] = fmaf(pw, bf16lo(x.y), a8[2]);
-            a8[3] = fmaf(pw, bf16hi(x.y), a8[3]);
-            a8[4] = fmaf(pw, bf16lo(x.z), a8[4]);
-            a8[5] = fmaf(pw, bf16hi(x.z), a8[5]);
-            a8[6] = fmaf(pw, bf16lo(x.w), a8[6]);
-            a8[7] = fmaf(pw, bf16hi(x.w), a8[7]);
+            const uint4 x = raw[r][cc];
+            vf[8 * cc + 0] = bf16lo(x.x); vf[8 * cc + 1] = bf16hi(x.x);
+            vf[8 * cc + 2] = bf16lo(x.y); vf[8 * cc + 3] = bf16hi(x.y);
+            vf[8 * cc + 4] = bf16lo(x.z); vf[8 * cc + 5] = bf16hi(x.z);
+            vf[8 * cc + 6] = bf16lo(x.w); vf[8 * cc + 7] = bf16hi(x.w);
+          }
+#pragma unroll
+          for (int a = 0; a < 4; ++a) {
+            const bool in = sc[r][a] != -INFINITY;
+            const float pw = in ? exp2f((sc[r][a] - m[a]) * kLog2e) : 0.f;
+            l[a] += pw;
+            cnt[a] += in ? 1 : 0;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) acc[a][e] = fmaf(pw, vf[e], acc[a][e]);
           }
         }
       }
-    }
-    sm100::named_bar(kBar, kComputeThreads);      // lists read before they refill
-    my_cnt = 0;
-  };
+    };
 
-  bool bad = false;
-  int committed = 0;                   // chunks whose MMAs thread 0 committed
-  if (tid == 0) {
-    if (issue_chunk(0)) committed = 1;
-    else { fail(p, hdr); bad = true; }
-  }
-  if (warp == 0) bad = __shfl_sync(0xffffffffu, bad ? 1 : 0, 0) != 0;
-
-  for (int c = 0; c < n_chunks; ++c) {
-    if (tid == 0 && !bad && c + 1 < n_chunks) {
-      if (issue_chunk(c + 1)) committed = c + 2;
-      else { fail(p, hdr); bad = true; }
-    }
-    if (warp == 0) bad = __shfl_sync(0xffffffffu, bad ? 1 : 0, 0) != 0;
-    if (!bad && !warp_wait(&hdr->mma_done[c & 1], (c >> 1) & 1)) {
-      if (lane == 0) fail(p, hdr);
-      bad = true;
-    }
-    sm100::tc_fence_after();
-    const int half = warp >> 2, quarter = warp & 3;
-    const bool has_tile = 2 * c + half < n_tiles;
-    const int kpos = half * kTileKeys + quarter * 32 + lane;
-    const int64_t t = t_begin + static_cast<int64_t>(c) * kChunkKeys + kpos;
-    const bool valid = !bad && has_tile && t < t_end;
-    float A[kN];
-#pragma unroll
-    for (int g = 0; g < kN; ++g) A[g] = 0.f;
-    if (!bad && has_tile)
-      sm100::tmem_ld16(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                           (c & 1) * 2 * kN + half * kN, A);
-    sm100::tc_fence_before();
-#pragma unroll
-    for (int g = 0; g < kN; ++g) A[g] = A[g] * p.scale;
-
-    bool over = false;
-    if (mode == kModeDump) {
-      if (valid) {
-#pragma unroll
-        for (int g = 0; g < GP; ++g)
-          if (g < G) p.scores_out[row0 + g * p.row_stride + t] = A[g];
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+      Unit un;
+      if (!unit_at(p, u, false, un)) continue;
+      const int j0 = un.kh * G;
+      const int64_t row0 = static_cast<int64_t>(un.b * p.h_q + j0) * p.row_stride;
+      if (MODE == kModeStep) {
+        if (widx == 0 && lane < kN)
+          h->tau[lane] = lane < G ? p.tau[un.b * p.h_q + j0 + lane] : INFINITY;
+        workers_sync<D>();
       }
-      if (p.hist != nullptr) {
-        // top byte of each score's order key, one shared atomic per distinct
-        // bin in the warp
-        uint32_t(*hs)[256] = reinterpret_cast<uint32_t(*)[256]>(smem + Lo::off_key);
 #pragma unroll
-        for (int g = 0; g < GP; ++g) {
-          const bool in = valid && g < G;
-          const uint32_t active = __ballot_sync(0xffffffffu, in);
-          if (in) {
-            const uint32_t bin = order_key(A[g]) >> 24;
-            const uint32_t peers = __match_any_sync(active, bin);
-            if (lane == __ffs(peers) - 1) atomicAdd(&hs[g][bin], static_cast<uint32_t>(__popc(peers)));
+      for (int a = 0; a < 4; ++a) {
+        m[a] = -INFINITY; l[a] = 0.f; cnt[a] = 0;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc[a][e] = 0.f;
+      }
+      vrow = static_cast<const uint16_t *>(p.V) + un.b * p.v_sb +
+             static_cast<int64_t>(un.kh * vpg + vsl) * p.v_sh;
+      int n_mine = 0;
+
+      const int first = (rank - static_cast<int>(g % C::kRanks) + C::kRanks) % C::kRanks;
+      for (int i = first; i < un.n_tiles; i += C::kRanks) {
+        const uint32_t gg = g + i;
+        const int tb = gg % C::kTBufs;
+        if (!warp_wait_bar(&h->tfull[tb], (gg / C::kTBufs) & 1, h)) {
+          if (lane == 0) fail(p, h);
+          bad = true;
+          break;
+        }
+        sm100::tc_fence_after();
+        float A[kN];
+        sm100::tmem_ld16(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + tb * kN, A);
+        sm100::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) sm100::mbar_arrive(&h->tempty[tb]);
+
+        const int64_t t0 = un.t_begin + static_cast<int64_t>(i) * kTileKeys + quarter * 32;
+        const int64_t t = t0 + lane;
+        const bool valid = t < un.t_end;
+
+        if (MODE == kModeDump) {
+#pragma unroll
+          for (int a = 0; a < kN; ++a) {
+            const float x = A[a] * p.scale;
+            if (valid && a < G) p.scores_out[row0 + a * p.row_stride + t] = x;
+            if (p.hist != nullptr) {
+              // top byte of the score's order key, one shared atomic per
+              // distinct bin in the warp
+              const bool in = valid && a < G;
+              const uint32_t active = __ballot_sync(0xffffffffu, in);
+              if (in) {
+                const uint32_t bin = order_key(x) >> 24;
+                const uint32_t peers = __match_any_sync(active, bin);
+                if (lane == __ffs(peers) - 1)
+                  atomicAdd(reinterpret_cast<uint32_t *>(scratch) + a * 256 + bin,
+                            static_cast<uint32_t>(__popc(peers)));
+              }
+            }
+          }
+          continue;
+        }
+
+        // ---- compare: the heads that keep this lane's key --------------------
+        float *rows = rows_base + (n_mine & 1) * 32 * kN;
+        ++n_mine;
+        uint32_t sel = 0;
+        {
+          const float4 *tq = reinterpret_cast<const float4 *>(h->tau);
+#pragma unroll
+          for (int a4 = 0; a4 < kN / 4; ++a4) {
+            const float4 tv = tq[a4];
+            const float tt[4] = {tv.x, tv.y, tv.z, tv.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int a = 4 * a4 + e;
+              const float x = A[a] * p.scale;
+              const bool keep = valid && x >= tt[e];
+              sel |= static_cast<uint32_t>(keep) << a;
+              A[a] = keep ? x : -INFINITY;
+            }
           }
         }
-      }
-    } else {
-      uint32_t selbits = 0;
+        if (sel != 0u) {
 #pragma unroll
-      for (int g = 0; g < GP; ++g) {
-        const bool sel = valid && g < G && A[g] >= tau_s[g];
-        const uint32_t bal = __ballot_sync(0xffffffffu, sel);
-        const int before = __shfl_sync(0xffffffffu, my_cnt, g);
-        if (sel) {
-          const int off = before + __popc(bal & lt_mask);
-          lkey[g][warp][off] = static_cast<int>(t - t_begin);
-          lsc[g][warp][off] = A[g];
+          for (int a4 = 0; a4 < kN / 4; ++a4)
+            *reinterpret_cast<float4 *>(rows + score_slot(lane, 4 * a4)) =
+                make_float4(A[4 * a4], A[4 * a4 + 1], A[4 * a4 + 2], A[4 * a4 + 3]);
         }
-        if (lane == g) my_cnt += __popc(bal);
-        selbits |= static_cast<uint32_t>(sel) << g;
+        if (p.sel_mask != nullptr && valid) {
+          for (int a = 0; a < G; ++a)
+            p.sel_mask[row0 + a * p.row_stride + t] = static_cast<uint8_t>((sel >> a) & 1u);
+        }
+        uint32_t mine = 0;
+#pragma unroll
+        for (int vv = 0; vv < 4; ++vv) {
+          const uint32_t bl = __ballot_sync(0xffffffffu, (sel & hm.smask[vv]) != 0u);
+          if (v == vv) mine = bl;
+        }
+        __syncwarp();
+        gather(mine, t0, un.t_begin, rows);
+        __syncwarp();            // rows read before a later tile overwrites them
       }
-      if (p.sel_mask != nullptr && valid) {
-        for (int g = 0; g < G; ++g)
-          p.sel_mask[row0 + g * p.row_stride + t] = static_cast<uint8_t>((selbits >> g) & 1u);
+      g += un.n_tiles;
+
+      // ---- end of unit -------------------------------------------------------
+      if (workers_any<D>(bad || aborted(h))) { bad = true; break; }
+      if (MODE == kModeDump) {
+        if (p.hist != nullptr) {
+          uint32_t *hs = reinterpret_cast<uint32_t *>(scratch);
+          for (int i = widx * 32 + lane; i < kN * 256; i += C::kWorkers * 32) {
+            const uint32_t c = hs[i];
+            if (c != 0u && i / 256 < G)
+              atomicAdd(&p.hist[static_cast<int64_t>(un.b * p.h_q + j0 + i / 256) * 256 + (i % 256)], c);
+            hs[i] = 0u;
+          }
+          workers_sync<D>();
+        }
+        continue;
       }
-      // one more chunk may add 32 keys per (head, warp)
-      over = __any_sync(0xffffffffu, my_cnt > C::kCap - 32);
+      // merge: every worker's 16 head states into shared memory, then
+      // per head the weights e^{m_w - m} of the workers, then the records
+      {
+        float *st = scratch + widx * C::kStateFloats;
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+          put_state<EPL>(st + (v * 4 + a) * C::kRec, c8, m[a], l[a], cnt[a], acc[a]);
+      }
+      workers_sync<D>();
+      float *wts = scratch + C::kWorkers * C::kStateFloats;       // [kN][kWorkers]
+      const int tw = widx * 32 + lane;
+      if (tw < kN) {
+        const int slot = tw, sv = slot >> 2, sa = slot & 3;
+        float mm = -INFINITY;
+        for (int w = 0; w < C::kWorkers; ++w) mm = fmaxf(mm, scratch[w * C::kStateFloats + slot * C::kRec]);
+        float ll = 0.f;
+        int nn = 0;
+        for (int w = 0; w < C::kWorkers; ++w) {
+          const float *r = scratch + w * C::kStateFloats + slot * C::kRec;
+          const float wt = r[0] == -INFINITY ? 0.f : exp2f((r[0] - mm) * kLog2e);
+          wts[slot * C::kWorkers + w] = wt;
+          ll = fmaf(wt, r[1], ll);
+          nn += __float_as_int(r[2]);
+        }
+        if (sa < pick4(hm.nh, sv)) {
+          const int j = j0 + pick4(hm.hbase, sv) + sa;
+          float *rec = p.partials + (static_cast<int64_t>(un.b * p.h_q + j) * p.S + un.s) * C::kRec;
+          rec[0] = mm;
+          rec[1] = ll;
+          rec[2] = __int_as_float(nn);
+          rec[3] = 0.f;
+        }
+      }
+      workers_sync<D>();
+      for (int idx = tw; idx < kN * D; idx += C::kWorkers * 32) {
+        const int slot = idx / D, dd = idx % D, sv = slot >> 2, sa = slot & 3;
+        if (sa >= pick4(hm.nh, sv)) continue;
+        float a = 0.f;
+        for (int w = 0; w < C::kWorkers; ++w)
+          a = fmaf(wts[slot * C::kWorkers + w],
+                   scratch[w * C::kStateFloats + slot * C::kRec + kRecPad + dd], a);
+        const int j = j0 + pick4(hm.hbase, sv) + sa;
+        p.partials[(static_cast<int64_t>(un.b * p.h_q + j) * p.S + un.s) * C::kRec + kRecPad + dd] = a;
+      }
+      workers_sync<D>();          // scratch read before the next unit reuses it
     }
-    // every warp has read this chunk's TMEM before thread 0 reuses the set
-    const bool any_bad = bar_any(bad);
-    if (any_bad) { bad = true; break; }
-    if (bar_any(over)) gather();
   }
-  if (!bad && mode != kModeDump) gather();
 
   // ---- teardown: every MMA has landed before TMEM is freed -----------------
-  if (tid == 0 && bad && committed > 0)
-    sm100::mbar_wait(&hdr->mma_done[(committed - 1) & 1], ((committed - 1) >> 1) & 1);
   sm100::tc_fence_before();
-  sm100::named_bar(kBar, kComputeThreads);
-  if (warp == 0) {
+  __syncthreads();
+  if (warp == 1) {
     sm100::tc_fence_after();
-    sm100::tmem_dealloc(tmem_base, kTmemCols);
-  }
-  if (mode == kModeDump) {
-    if (p.hist != nullptr && !bad && !aborted(hdr)) {
-      const uint32_t *hs = reinterpret_cast<const uint32_t *>(smem + Lo::off_key);
-      for (int i = tid; i < G * 256; i += kComputeThreads) {
-        const uint32_t v = hs[i];
-        if (v != 0u) atomicAdd(&p.hist[static_cast<int64_t>(b * p.h_q + j0 + i / 256) * 256 + (i % 256)], v);
-      }
-    }
-    return;
-  }
-  if (bad || aborted(hdr)) return;
-
-  // ---- merge the two halves of each head and write the split's record -----
-  // (the K stages are idle now: every tile landed and was consumed)
-  float *mrg = reinterpret_cast<float *>(stages);      // [kN][D + 4]
-  if (part == 1 && live) {
-    float *r = mrg + gh * (D + kRecPad);
-    if (c8 == 0) { r[0] = m_run; r[1] = l_run; r[2] = __int_as_float(cnt_run); }
-#pragma unroll
-    for (int cc = 0; cc < CPL; ++cc)
-#pragma unroll
-      for (int v = 0; v < 8; ++v) r[kRecPad + (c8 + 8 * cc) * 8 + v] = acc[8 * cc + v];
-  }
-  sm100::named_bar(kBar, kComputeThreads);
-  if (part == 0 && live) {
-    const float *r = mrg + gh * (D + kRecPad);
-    const float m1 = r[0], l1 = r[1];
-    const int n1 = __float_as_int(r[2]);
-    const float m = fmaxf(m_run, m1);
-    const float w0 = m_run == -INFINITY ? 0.f : exp2f((m_run - m) * kLog2e);
-    const float w1 = m1 == -INFINITY ? 0.f : exp2f((m1 - m) * kLog2e);
-    float *rec = p.partials + (static_cast<int64_t>(b * p.h_q + j0 + gh) * p.S + s) * (D + kRecPad);
-    if (c8 == 0) {
-      rec[0] = m;
-      rec[1] = w0 * l_run + w1 * l1;
-      rec[2] = __int_as_float(cnt_run + n1);
-      rec[3] = 0.f;
-    }
-#pragma unroll
-    for (int cc = 0; cc < CPL; ++cc)
-#pragma unroll
-      for (int v = 0; v < 8; ++v) {
-        const int i = (c8 + 8 * cc) * 8 + v;
-        rec[kRecPad + i] = w0 * acc[8 * cc + v] + w1 * r[kRecPad + i];
-      }
+    sm100::tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
 
@@ -484,52 +623,111 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-template <int D, int GP>
-cudaError_t launch_tc(const StepParams &p, int mode, const CUtensorMap &map, cudaStream_t st) {
+constexpr int kMaxDevices = 64;
+
+// SM count of a device, cached per device.
+int sm_count(int dev) {
+  static std::atomic<int> cache[kMaxDevices];
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      return -1;
+    cache[dev].store(n, std::memory_order_relaxed);
+  }
+  return n;
+}
+
+template <int D, int MODE>
+cudaError_t launch_tc(const StepParams &p, const CUtensorMap &kmap, const CUtensorMap &qmap,
+                      const HeadMap &hm, int dev, cudaStream_t st) {
   using Lo = Layout<D>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(saga_tc_kernel<D, GP>,
+  static std::atomic<bool> attr_set[kMaxDevices];
+  if (!attr_set[dev].load(std::memory_order_acquire)) {
+    cudaError_t e = cudaFuncSetAttribute(saga_tc_kernel<D, MODE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Lo::alloc);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
-  dim3 grid(p.S, p.B * p.h_k);
-  saga_tc_kernel<D, GP><<<grid, kThreads, Lo::alloc, st>>>(p, mode, map);
+  const int sms = sm_count(dev);
+  if (sms < 1) return cudaErrorInvalidDevice;
+  const int n_units = p.B * p.h_k * p.S;
+  const int grid = n_units < sms ? n_units : sms;
+  if (grid < 1) return cudaSuccess;
+  saga_tc_kernel<D, MODE><<<grid, Cfg<D>::kThreads, Lo::alloc, st>>>(p, kmap, qmap, hm);
   return cudaGetLastError();
 }
 
-template <int D>
-cudaError_t launch_tc_d(const StepParams &p, int mode, int gp, const CUtensorMap &map,
-                        cudaStream_t st) {
-  switch (gp) {
-    case 4: return launch_tc<D, 4>(p, mode, map, st);
-    case 8: return launch_tc<D, 8>(p, mode, map, st);
-    case 12: return launch_tc<D, 12>(p, mode, map, st);
-    case 16: return launch_tc<D, 16>(p, mode, map, st);
-    default: return cudaErrorInvalidValue;
+// Lane groups: value head slot vs = v / chunks, chunk c = v % chunks of that
+// value head's h_q / h_v query heads (four per chunk).
+bool make_head_map(int h_q, int h_k, int h_v, HeadMap &hm) {
+  if (h_k < 1 || h_v < 1 || h_q % h_v != 0 || h_v % h_k != 0) return false;
+  const int G = h_q / h_k, hpv = h_q / h_v, vpg = h_v / h_k;
+  const int chunks = (hpv + 3) / 4;
+  if (G > kN || vpg * chunks > 4) return false;
+  for (int v = 0; v < 4; ++v) {
+    const int vs = v / chunks, c = v % chunks;
+    if (vs < vpg && c * 4 < hpv) {
+      hm.hbase[v] = vs * hpv + c * 4;
+      hm.nh[v] = hpv - c * 4 < 4 ? hpv - c * 4 : 4;
+      hm.vs[v] = vs;
+    } else {
+      hm.hbase[v] = 0;
+      hm.nh[v] = 0;
+      hm.vs[v] = 0;
+    }
+    hm.smask[v] = ((1u << hm.nh[v]) - 1u) << hm.hbase[v];
   }
+  return true;
 }
 
 }  // namespace
 
-cudaError_t launch_saga_tc(const StepParams &p, int mode, int d, int gp, cudaStream_t st) {
+bool saga_tc_supports(int dtype, int d, int h_q, int h_k, int h_v) {
+  HeadMap hm;
+  return dtype == SAGA_BF16 && (d == 64 || d == 128) && make_head_map(h_q, h_k, h_v, hm);
+}
+
+cudaError_t launch_saga_tc(const StepParams &p, int mode, int d, cudaStream_t st) {
+  HeadMap hm;
+  if (!make_head_map(p.h_q, p.h_k, p.h_v, hm)) return cudaErrorInvalidValue;
+  if (mode != kModeDump && mode != kModeStep) return cudaErrorInvalidValue;
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return cudaErrorNotSupported;
-  CUtensorMap map;
-  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(p.cap),
-                              static_cast<cuuint64_t>(p.h_k), static_cast<cuuint64_t>(p.B)};
-  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2,
-                                 static_cast<cuuint64_t>(p.k_sh) * 2,
-                                 static_cast<cuuint64_t>(p.k_sb) * 2};
-  const cuuint32_t box[4] = {64, kTileKeys, 1, 1};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   const cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(p.K), dims,
-                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  if (d == 64) return launch_tc_d<64>(p, mode, gp, map, st);
-  if (d == 128) return launch_tc_d<128>(p, mode, gp, map, st);
+  CUtensorMap kmap, qmap;
+  {
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(p.cap),
+                                static_cast<cuuint64_t>(p.h_k), static_cast<cuuint64_t>(p.B)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2,
+                                   static_cast<cuuint64_t>(p.k_sh) * 2,
+                                   static_cast<cuuint64_t>(p.k_sb) * 2};
+    const cuuint32_t box[4] = {64, kTileKeys, 1, 1};
+    if (enc(&kmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(p.K), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(p.h_q),
+                                static_cast<cuuint64_t>(p.B)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(p.q_sh) * 2,
+                                   static_cast<cuuint64_t>(p.q_sb) * 2};
+    const cuuint32_t box[3] = {64, kN, 1};
+    if (enc(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(p.q), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  if (d == 64)
+    return mode == kModeDump ? launch_tc<64, kModeDump>(p, kmap, qmap, hm, dev, st)
+                             : launch_tc<64, kModeStep>(p, kmap, qmap, hm, dev, st);
+  if (d == 128)
+    return mode == kModeDump ? launch_tc<128, kModeDump>(p, kmap, qmap, hm, dev, st)
+                             : launch_tc<128, kModeStep>(p, kmap, qmap, hm, dev, st);
   return cudaErrorInvalidValue;
 }
 
