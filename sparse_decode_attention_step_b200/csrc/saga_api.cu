@@ -14,7 +14,8 @@ namespace {
 
 constexpr int64_t kSms = 148;              // B200 SMs: the persistent grid
 constexpr int64_t kTileKeys = 128;         // split lengths are multiples of a K tile
-constexpr int64_t kUnitTiles = 32;         // at most about this many tiles per split
+constexpr int64_t kUnitTiles = 32;         // grid-per-split kernels: at most about this many tiles per split
+constexpr int64_t kPersistTiles = 128;     // persistent kernel: at most about this many tiles per unit
 constexpr size_t kAlign = 256;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -26,16 +27,27 @@ struct Plan {
   size_t off_partials, off_scores, off_hist, total;
 };
 
-// Splits of equal length (a multiple of the K tile) such that the
-// (b, kh, split) units number about a whole multiple of the SM count, with at
-// most about kUnitTiles tiles each.
-Plan make_plan(const saga_shape &s) {
+bool use_tc(const saga_shape &s);
+
+// Splits of equal length, a multiple of the K tile.
+// Grid-per-split kernels (SIMT, dense): the (b, kh, split) units number about a
+// whole multiple of the SM count, with at most about kUnitTiles tiles each.
+// Persistent tensor-core kernel: at most one unit per SM and wave, units of up
+// to about kPersistTiles tiles, since every unit ends with a merge of the
+// workers' states.
+Plan make_plan(const saga_shape &s, bool persistent) {
   Plan p{};
   const int64_t rows = static_cast<int64_t>(s.B) * s.h_k;
   const int64_t L = std::max<int64_t>(1, s.max_l_kv);
   const int64_t tiles = rows * ceil_div(L, kTileKeys);
-  const int64_t waves = std::max<int64_t>(1, ceil_div(tiles, kSms * kUnitTiles));
-  const int64_t s_target = std::max<int64_t>(1, ceil_div(kSms * waves, rows));
+  int64_t s_target;
+  if (persistent) {
+    const int64_t waves = std::max<int64_t>(1, ceil_div(tiles, kSms * kPersistTiles));
+    s_target = std::max<int64_t>(1, kSms * waves / rows);
+  } else {
+    const int64_t waves = std::max<int64_t>(1, ceil_div(tiles, kSms * kUnitTiles));
+    s_target = std::max<int64_t>(1, ceil_div(kSms * waves, rows));
+  }
   p.split_len = ceil_div(ceil_div(L, s_target), kTileKeys) * kTileKeys;
   p.S = static_cast<int>(ceil_div(L, p.split_len));
   const size_t rec = static_cast<size_t>(s.d + kRecPad) * sizeof(float);
@@ -44,6 +56,14 @@ Plan make_plan(const saga_shape &s) {
   p.off_hist = align_up(p.off_scores + static_cast<size_t>(s.B) * s.h_q * s.max_l_kv * sizeof(float));
   p.total = align_up(p.off_hist + static_cast<size_t>(s.B) * s.h_q * 256 * sizeof(uint32_t));
   return p;
+}
+
+// The plan of the SAGA calls (step, refresh, debug scores) of a shape.
+Plan saga_plan(const saga_shape &s) { return make_plan(s, use_tc(s)); }
+
+// One workspace serves every call of a shape: the larger of the two plans.
+size_t workspace_bytes(const saga_shape &s) {
+  return std::max(make_plan(s, true).total, make_plan(s, false).total);
 }
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -71,7 +91,7 @@ saga_status check_shape(const saga_shape *s) {
 
 saga_status check_ws(const saga_shape &s, void *ws, size_t ws_bytes) {
   if (ws == nullptr || !aligned(ws, kAlign)) return SAGA_ERR_WORKSPACE;
-  if (ws_bytes < make_plan(s).total) return SAGA_ERR_WORKSPACE;
+  if (ws_bytes < workspace_bytes(s)) return SAGA_ERR_WORKSPACE;
   return SAGA_OK;
 }
 
@@ -129,7 +149,7 @@ saga_status run_step(const saga_shape &s, const Plan &pl, StepParams p, int mode
 }  // namespace
 
 // Scratch a plain step needs (error word + per-split states; no score rows).
-size_t plain_step_scratch_bytes(const saga_shape &s) { return make_plan(s).off_scores; }
+size_t plain_step_scratch_bytes(const saga_shape &s) { return saga_plan(s).off_scores; }
 
 // saga_decode_step's checks and launches with a caller-chosen scratch buffer
 // in place of the workspace (sel_mask not supported).
@@ -146,7 +166,7 @@ saga_status plain_step_with_scratch(const saga_shape *shape, const void *q, cons
     return SAGA_ERR_INVALID_ARG;
   if (scratch == nullptr || !aligned(scratch, kAlign) || scratch_bytes < plain_step_scratch_bytes(s))
     return SAGA_ERR_WORKSPACE;
-  const Plan pl = make_plan(s);
+  const Plan pl = saga_plan(s);
   StepParams p = base_params(s, pl, q, K, V, l_kv, scratch);
   p.tau = tau;
   return run_step(s, pl, p, kModeStep, out, sel_count, st);
@@ -172,7 +192,7 @@ void saga_shape_contiguous(saga_shape *s, int32_t B, int32_t h_q, int32_t h_k, i
 size_t saga_workspace_size(const saga_shape *shape, int32_t N) {
   (void)N;
   if (check_shape(shape) != SAGA_OK) return 0;
-  return make_plan(*shape).total;
+  return workspace_bytes(*shape);
 }
 
 saga_status saga_workspace_init(void *ws, size_t ws_bytes, saga_stream_t stream) {
@@ -192,7 +212,7 @@ saga_status saga_decode_step(const saga_shape *shape, const void *q, const void 
       !aligned(tau, 4) || !aligned(out, 16) || (sel_count && !aligned(sel_count, 4)))
     return SAGA_ERR_INVALID_ARG;
   if ((r = check_ws(s, ws, ws_bytes)) != SAGA_OK) return r;
-  const Plan pl = make_plan(s);
+  const Plan pl = saga_plan(s);
   StepParams p = base_params(s, pl, q, K, V, l_kv, ws);
   p.tau = tau;
   p.sel_mask = sel_mask;
@@ -215,7 +235,7 @@ saga_status saga_refresh_threshold(const saga_shape *shape, const void *q, const
     return SAGA_ERR_INVALID_ARG;
   if ((r = check_ws(s, ws, ws_bytes)) != SAGA_OK) return r;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const Plan pl = make_plan(s);
+  const Plan pl = saga_plan(s);
   StepParams p = base_params(s, pl, q, K, V, l_kv, ws);
   float *rows = scores != nullptr
                     ? scores
@@ -262,7 +282,7 @@ saga_status gqa_dense_decode(const saga_shape *shape, const void *q, const void 
     return SAGA_ERR_INVALID_ARG;
   if ((r = check_ws(s, ws, ws_bytes)) != SAGA_OK) return r;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const Plan pl = make_plan(s);
+  const Plan pl = make_plan(s, false);
   StepParams p = base_params(s, pl, q, K, V, l_kv, ws);
   cudaError_t e = launch_dense_split(p, s.dtype, s.d, group_pad(s), st);
   if (e != cudaSuccess) return SAGA_ERR_CUDA;
@@ -280,7 +300,7 @@ saga_status saga_debug_scores(const saga_shape *shape, const void *q, const void
   if ((r = check_inputs(s, q, K, l_kv)) != SAGA_OK) return r;
   if (scores == nullptr || !aligned(scores, 4)) return SAGA_ERR_INVALID_ARG;
   if (ws == nullptr || !aligned(ws, kAlign) || ws_bytes < kAlign) return SAGA_ERR_WORKSPACE;
-  const Plan pl = make_plan(s);
+  const Plan pl = saga_plan(s);
   StepParams p = base_params(s, pl, q, K, nullptr, l_kv, ws);
   p.partials = nullptr;
   p.scores_out = scores;

@@ -376,7 +376,13 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
         float sc[kRows][4];
 #pragma unroll
         for (int r = 0; r < kRows; ++r) {
+          if (r0 + r >= nmax) {
+#pragma unroll
+            for (int a = 0; a < 4; ++a) sc[r][a] = -INFINITY;
+            continue;
+          }
           const int kk = mine != 0u ? __ffs(mine) - 1 : -1;
+
           mine &= mine - 1u;
           // idle slots re-read a row of the unit, which always exists
           const int64_t tr = kk >= 0 ? t0 + kk : t_any;
@@ -390,21 +396,32 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
             sc[r][a] = (kk >= 0 && a < nh) ? rows[score_slot(ks, hd)] : -INFINITY;
           }
         }
+        float mnew[4];
+        bool grow = false;
 #pragma unroll
         for (int a = 0; a < 4; ++a) {
           float mx = sc[0][a];
 #pragma unroll
           for (int r = 1; r < kRows; ++r) mx = fmaxf(mx, sc[r][a]);
-          const float mn = fmaxf(m[a], mx);
-          const float corr = mn == m[a] ? 1.f : exp2f((m[a] - mn) * kLog2e);
-          m[a] = mn;
-          l[a] *= corr;
-#pragma unroll
-          for (int e = 0; e < EPL; ++e) acc[a][e] *= corr;
+          mnew[a] = fmaxf(m[a], mx);
+          grow |= mnew[a] != m[a];
         }
+        if (__any_sync(0xffffffffu, grow)) {
+#pragma unroll
+          for (int a = 0; a < 4; ++a) {
+            const float corr = mnew[a] == m[a] ? 1.f : exp2f((m[a] - mnew[a]) * kLog2e);
+            m[a] = mnew[a];
+            l[a] *= corr;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) acc[a][e] *= corr;
+          }
+        }
+
 #pragma unroll
         for (int r = 0; r < kRows; ++r) {
+          if (r0 + r >= nmax) break;
           float vf[EPL];
+
 #pragma unroll
           for (int cc = 0; cc < CPL; ++cc) {
             const uint4 x = raw[r][cc];
@@ -416,7 +433,9 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
 #pragma unroll
           for (int a = 0; a < 4; ++a) {
             const bool in = sc[r][a] != -INFINITY;
+            if (!__any_sync(0xffffffffu, in)) continue;
             const float pw = in ? exp2f((sc[r][a] - m[a]) * kLog2e) : 0.f;
+
             l[a] += pw;
             cnt[a] += in ? 1 : 0;
 #pragma unroll
