@@ -14,6 +14,8 @@ Prints one JSON line (rank 0):
   roofline   the plain-step call (the dominant one): algorithmic bytes per
              call / its mean duration, against the measured HBM copy peak;
   dense_gqa  the library's dense GQA stack at the same shape, same metric;
+  saga_full  full attention over the same SAGA-headed caches (the ablation arm
+             between dense GQA and SAGA + Atop-N);
   cpu_baseline  the float64 oracle on the host cores, on a bounded sample.
 
 With --impl reference the oracle alone is timed (the reference arm).
@@ -363,6 +365,13 @@ class Stack:
         for l in range(self.nl):
             self.layer_call(t, l, refresh)
 
+    def full_step(self, t):
+        """Full attention over the same (SAGA-headed) caches, every layer."""
+        r = t % self.replicas
+        for l in range(self.nl):
+            self.saga.dense_decode(self.shape, self.q[l], self.K[r * self.nl + l],
+                                   self.V[r * self.nl + l], self.l, self.out[l], self.ws)
+
 
 def kernels_per_call(dense, refresh):
     if dense:
@@ -557,6 +566,47 @@ def run_ours(args, w):
         del stk_dense
         torch.cuda.empty_cache()
 
+    # ---- SAGA full attention on the same stack: the ablation's "SAGA, full" arm
+    full = None
+    if not args.no_dense and w.h_k != w.h_v:
+        st.q.copy_(Q[0])
+        for t in range(2):
+            st.full_step(t)
+        torch.cuda.synchronize()
+        barrier(world)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        nf = args.dense_steps
+
+        def full_steps():
+            for t in range(nf):
+                st.q.copy_(Q[t % T_total], non_blocking=True)
+                st.full_step(t)
+        if use_graph:
+            gf = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gf):
+                full_steps()
+            torch.cuda.synchronize()
+        else:
+            torch.cuda._sleep(int(2e8))
+        f0.record(stream)
+        if use_graph:
+            gf.replay()
+        else:
+            full_steps()
+        f1.record(stream)
+        torch.cuda.synchronize()
+        fms = max_over_ranks(f0.elapsed_time(f1), world)
+        fvalue = aggregate_value(nf, fms, world)
+        fbytes_step = w.layers * ((w.h_k + w.h_v) * float(np.sum(lens)) * d * esz + qo_bytes)
+        fgbs = fbytes_step / (fms / nf / 1e3) / 1e9
+        full = {"value": fvalue, "unit": "steps/s", "ms_per_step": fms / nf,
+                "tokens_per_s": fvalue * B, "achieved_gbs": fgbs, "frac_of_peak": fgbs / peak,
+                "h_k": w.h_k, "h_v": w.h_v, "steps": nf,
+                "speedup_saga_atopn_over_full": value / fvalue,
+                "speedup_full_over_dense_gqa": (fvalue / dense["value"]) if dense else None}
+        if use_graph:
+            del gf
+
     clocks = clk.summary()
     result = None
     if rank == 0:
@@ -594,6 +644,7 @@ def run_ours(args, w):
             "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "dense_gqa": dense,
+            "saga_full": full,
             "clocks": clocks,
             "cpu_baseline": cpu,
         }

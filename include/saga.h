@@ -152,12 +152,30 @@ saga_status saga_refresh_threshold(const saga_shape *shape, const void *q,
 
 /*
  * Full-attention GQA decode (Eq. 2-4 over every t < l_kv[b]): the dense
- * baseline the sparse step is measured against. Requires h_k == h_v.
+ * baseline the sparse step is measured against. Requires h_k == h_v and
+ * h_q / h_k <= 16 (else SAGA_ERR_INVALID_ARG / SAGA_ERR_UNSUPPORTED).
  */
 saga_status gqa_dense_decode(const saga_shape *shape, const void *q,
                              const void *K, const void *V,
                              const int32_t *l_kv, float *out, void *ws,
                              size_t ws_bytes, saga_stream_t stream);
+
+/*
+ * Full-attention decode with SAGA's asymmetric heads (SAGA Architecture;
+ * Eq. 2-4 over every t < l_kv[b], query head j reading key head
+ * floor(j*h_k/h_q) and value head floor(j*h_v/h_q)): the "SAGA, full
+ * attention" arm of the paper's ablation of key merging and Atop-N, and,
+ * with h_k == h_v, the same result as gqa_dense_decode.
+ *   Arguments, layouts, ownership and workspace as for gqa_dense_decode;
+ *   out [B][h_q][d] fp32 is written.
+ *   Supported: h_v / h_k == 1 with h_q / h_k <= 16, or h_v / h_k in {2, 4}
+ *   with h_q / h_k in {4, 8, 12, 16}; other shapes return
+ *   SAGA_ERR_UNSUPPORTED and nothing is enqueued.
+ */
+saga_status saga_dense_decode(const saga_shape *shape, const void *q,
+                              const void *K, const void *V,
+                              const int32_t *l_kv, float *out, void *ws,
+                              size_t ws_bytes, saga_stream_t stream);
 
 /*
  * saga_decode_step without a workspace argument, for callers that cannot
@@ -173,7 +191,7 @@ saga_status gqa_dense_decode(const saga_shape *shape, const void *q,
  *     shape needing more than SAGA_NOALLOC_SCRATCH_BYTES is rejected with
  *     SAGA_ERR_WORKSPACE, an invalid one with SAGA_ERR_INVALID_ARG, and
  *     nothing is enqueued then. (The 16-layer batch-8 128K workload needs
- *     2.6 MB per layer call.)
+ *     about 0.6 MB per layer call.)
  *   - It calls no cudaMalloc, cudaFree or other allocating routine.
  *   - The first call on each device looks up the array's device address
  *     with that device current; make that first call before any stream

@@ -55,6 +55,7 @@ _SIGS = {
     "saga_refresh_threshold": (ctypes.c_int, [_SP, _P, _P, _P, _P, ctypes.c_int32, _P, _P,
                                               _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "gqa_dense_decode": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "saga_dense_decode": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "saga_debug_scores": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "saga_decode_step_noalloc": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P, _P, _P]),
     "saga_read_device_error": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_int32)]),
@@ -160,6 +161,14 @@ def gqa_dense_decode(shp, q, K, V, l_kv, out, ws, stream=None):
     p, n = _ws(ws)
     _check(load().gqa_dense_decode(ctypes.byref(shp), _ptr(q), _ptr(K), _ptr(V), _ptr(l_kv),
                                    _ptr(out), p, n, _stream(stream)), "gqa_dense_decode")
+
+
+def dense_decode(shp, q, K, V, l_kv, out, ws, stream=None):
+    """Full attention with the shape's key and value head maps (SAGA full
+    attention when h_k < h_v, GQA full attention when h_k == h_v)."""
+    p, n = _ws(ws)
+    _check(load().saga_dense_decode(ctypes.byref(shp), _ptr(q), _ptr(K), _ptr(V), _ptr(l_kv),
+                                    _ptr(out), p, n, _stream(stream)), "saga_dense_decode")
 
 
 NOALLOC_SCRATCH_BYTES = 4 << 20

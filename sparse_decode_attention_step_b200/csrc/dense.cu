@@ -1,10 +1,12 @@
-// Dense GQA decode split kernel: the full-attention baseline, Eq. (2-4) over
-// every position. One CTA per (b, kv head, split of l_kv). Each sub-chunk of
-// 256 positions is scored (one position per thread, all G query heads of the
-// group), the chunk maximum updates the running softmax state, and the
-// probabilities weight the V rows (one V row per warp-iteration, d split
-// across the lanes). The per-split states go to the same combine kernel as
-// the sparse step.
+// Dense decode split kernel: full attention, Eq. (2-4) over every position,
+// for GQA (h_k == h_v) and for SAGA's asymmetric heads (h_k < h_v: the G query
+// heads of a key head read VPG value heads, G / VPG query heads each). One CTA
+// per (b, key head, split of l_kv). Each sub-chunk of 256 positions is scored
+// (one position per thread, all G query heads of the group), the chunk
+// maximum updates the running softmax state, and the probabilities weight the
+// V rows (the VPG rows of one position per warp-iteration, d split across the
+// lanes). The per-split states go to the same combine kernel as the sparse
+// step.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -70,13 +72,14 @@ __device__ __forceinline__ void vslice(const uint16_t *row, int lane, float (&v)
   }
 }
 
-template <typename T, int D, int GP>
+template <typename T, int D, int GP, int VPG>
 __global__ void __launch_bounds__(kThreads) dense_split_kernel(const StepParams p) {
   constexpr int VPL = D / 32;
+  constexpr int HPV = GP / VPG;              // query heads per value head (VPG > 1: GP == G)
   __shared__ __align__(16) float qs[D * GP];
   __shared__ __align__(16) float ps[kChunk][GP];
   __shared__ float red[kWarps][GP];
-  __shared__ float red_acc[kWarps][GP][D];
+  __shared__ float red_acc[kWarps][4][D];      // four heads at a time
   __shared__ float red_l[kWarps][GP];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -97,7 +100,7 @@ __global__ void __launch_bounds__(kThreads) dense_split_kernel(const StepParams 
   __syncthreads();
 
   const T *krow0 = static_cast<const T *>(p.K) + b * p.k_sb + kh * p.k_sh;
-  const T *vrow0 = static_cast<const T *>(p.V) + b * p.v_sb + kh * p.v_sh;
+  const T *vrow0 = static_cast<const T *>(p.V) + b * p.v_sb + (kh * VPG) * p.v_sh;
 
   float m_run[GP], l_run[GP], acc[GP][VPL];
 #pragma unroll
@@ -140,8 +143,9 @@ __global__ void __launch_bounds__(kThreads) dense_split_kernel(const StepParams 
     __syncthreads();
     const int n = static_cast<int>(t_end - base < kChunk ? t_end - base : kChunk);
     for (int kk = warp; kk < n; kk += kWarps) {
-      float vv[VPL];
-      vslice<VPL>(vrow0 + (base + kk) * D, lane, vv);
+      float vv[VPG][VPL];
+#pragma unroll
+      for (int vs = 0; vs < VPG; ++vs) vslice<VPL>(vrow0 + vs * p.v_sh + (base + kk) * D, lane, vv[vs]);
       const float4 *pv = reinterpret_cast<const float4 *>(&ps[kk][0]);
 #pragma unroll
       for (int g4 = 0; g4 < GP / 4; ++g4) {
@@ -149,67 +153,95 @@ __global__ void __launch_bounds__(kThreads) dense_split_kernel(const StepParams 
         const float pw[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          l_run[4 * g4 + u] += pw[u];
+          const int g = 4 * g4 + u;
+          l_run[g] += pw[u];
 #pragma unroll
-          for (int v = 0; v < VPL; ++v)
-            acc[4 * g4 + u][v] = fmaf(pw[u], vv[v], acc[4 * g4 + u][v]);
+          for (int v = 0; v < VPL; ++v) acc[g][v] = fmaf(pw[u], vv[g / HPV][v], acc[g][v]);
         }
       }
     }
     __syncthreads();
   }
 
-  // Every warp holds the same m_run; sum the warps' l and acc.
+  // Every warp holds the same m_run; sum the warps' l and acc, four heads at a time.
   if (tid == 0) {
 #pragma unroll
     for (int g = 0; g < GP; ++g) red[0][g] = m_run[g];
   }
 #pragma unroll
-  for (int g = 0; g < GP; ++g) {
-#pragma unroll
-    for (int v = 0; v < VPL; ++v) red_acc[warp][g][lane * VPL + v] = acc[g][v];
+  for (int g = 0; g < GP; ++g)
     if (lane == 0) red_l[warp][g] = l_run[g];
-  }
-  __syncthreads();
-  for (int idx = tid; idx < G * D; idx += kThreads) {
-    const int g = idx / D, i = idx % D;
-    float a = 0.f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) a += red_acc[w][g][i];
-    float *rec = p.partials + (static_cast<int64_t>(b * p.h_q + j0 + g) * p.S + s) * (D + kRecPad);
-    rec[kRecPad + i] = a;
-    if (i == 0) {
-      float l = 0.f;
+  for (int g0 = 0; g0 < GP; g0 += 4) {
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) l += red_l[w][g];
-      rec[0] = red[0][g];
-      rec[1] = l;
-      rec[2] = __int_as_float(static_cast<int>(t_end - t_begin));
-      rec[3] = 0.f;
+    for (int gg = 0; gg < 4; ++gg)
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) red_acc[warp][gg][lane * VPL + v] = acc[g0 + gg][v];
+    __syncthreads();
+    for (int idx = tid; idx < 4 * D; idx += kThreads) {
+      const int g = g0 + idx / D, i = idx % D;
+      if (g >= G) continue;
+      float a = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) a += red_acc[w][idx / D][i];
+      float *rec = p.partials + (static_cast<int64_t>(b * p.h_q + j0 + g) * p.S + s) * (D + kRecPad);
+      rec[kRecPad + i] = a;
+      if (i == 0) {
+        float l = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) l += red_l[w][g];
+        rec[0] = red[0][g];
+        rec[1] = l;
+        rec[2] = __int_as_float(static_cast<int>(t_end - t_begin));
+        rec[3] = 0.f;
+      }
     }
+    __syncthreads();
   }
 }
 
 }  // namespace
 
-template <typename T, int D>
-static cudaError_t launch_dd(const StepParams &p, int gp, dim3 grid, cudaStream_t st) {
+template <typename T, int D, int VPG>
+static cudaError_t launch_dv(const StepParams &p, int gp, dim3 grid, cudaStream_t st) {
   switch (gp) {
-    case 4: dense_split_kernel<T, D, 4><<<grid, kThreads, 0, st>>>(p); break;
-    case 8: dense_split_kernel<T, D, 8><<<grid, kThreads, 0, st>>>(p); break;
+    case 4: dense_split_kernel<T, D, 4, VPG><<<grid, kThreads, 0, st>>>(p); break;
+    case 8: dense_split_kernel<T, D, 8, VPG><<<grid, kThreads, 0, st>>>(p); break;
+    case 12: dense_split_kernel<T, D, 12, VPG><<<grid, kThreads, 0, st>>>(p); break;
+    case 16: dense_split_kernel<T, D, 16, VPG><<<grid, kThreads, 0, st>>>(p); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
 }
 
-cudaError_t launch_dense_split(const StepParams &p, int dtype, int d, int gp, cudaStream_t st) {
+template <typename T, int D>
+static cudaError_t launch_dd(const StepParams &p, int gp, int vpg, dim3 grid, cudaStream_t st) {
+  switch (vpg) {
+    case 1: return launch_dv<T, D, 1>(p, gp, grid, st);
+    case 2: return launch_dv<T, D, 2>(p, gp, grid, st);
+    case 4: return launch_dv<T, D, 4>(p, gp, grid, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+bool dense_supports(int h_q, int h_k, int h_v) {
+  if (h_k < 1 || h_v % h_k != 0 || h_q % h_v != 0) return false;
+  const int G = h_q / h_k, vpg = h_v / h_k;
+  if (vpg == 1) return G <= 16;
+  return (vpg == 2 || vpg == 4) && (G == 4 || G == 8 || G == 12 || G == 16) && G % vpg == 0;
+}
+
+cudaError_t launch_dense_split(const StepParams &p, int dtype, int d, cudaStream_t st) {
+  if (!dense_supports(p.h_q, p.h_k, p.h_v)) return cudaErrorInvalidValue;
+  const int G = p.h_q / p.h_k, vpg = p.h_v / p.h_k;
+  const int gp = vpg == 1 ? (G + 3) / 4 * 4 : G;
   dim3 grid(p.S, p.B * p.h_k);
   if (dtype == SAGA_BF16) {
-    if (d == 64) return launch_dd<uint16_t, 64>(p, gp, grid, st);
-    if (d == 128) return launch_dd<uint16_t, 128>(p, gp, grid, st);
+    if (d == 64) return launch_dd<uint16_t, 64>(p, gp, vpg, grid, st);
+    if (d == 128) return launch_dd<uint16_t, 128>(p, gp, vpg, grid, st);
   } else {
-    if (d == 64) return launch_dd<float, 64>(p, gp, grid, st);
-    if (d == 128) return launch_dd<float, 128>(p, gp, grid, st);
+    if (d == 64) return launch_dd<float, 64>(p, gp, vpg, grid, st);
+    if (d == 128) return launch_dd<float, 128>(p, gp, vpg, grid, st);
   }
   return cudaErrorInvalidValue;
 }

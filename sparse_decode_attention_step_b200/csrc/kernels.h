@@ -35,8 +35,10 @@ cudaError_t launch_radix_select(const float *scores, int64_t row_stride, const i
                                 int N, float *tau, int B, int h_q, int64_t cap, int64_t max_l_kv,
                                 const uint32_t *hist0, cudaStream_t st);
 
-// Dense GQA split kernel over grid (S, B * h_k), h_k == h_v; gp = h_q / h_k rounded up to 4.
-cudaError_t launch_dense_split(const StepParams &p, int dtype, int d, int gp, cudaStream_t st);
+// Dense (full-attention) split kernel over grid (S, B * h_k): GQA (h_k == h_v,
+// h_q / h_k <= 16) or SAGA heads (h_v / h_k in {2, 4}, h_q / h_k in {4, 8, 12, 16}).
+bool dense_supports(int h_q, int h_k, int h_v);
+cudaError_t launch_dense_split(const StepParams &p, int dtype, int d, cudaStream_t st);
 
 // Plain step with a caller-chosen scratch buffer (see saga_decode_step_noalloc).
 size_t plain_step_scratch_bytes(const saga_shape &s);

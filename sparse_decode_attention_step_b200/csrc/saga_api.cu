@@ -146,6 +146,26 @@ saga_status run_step(const saga_shape &s, const Plan &pl, StepParams p, int mode
   return cuda_status(e);
 }
 
+// Full attention (Eq. 2-4) with the shape's key and value head maps: the
+// dense kernel, then the combine.
+saga_status run_dense(const saga_shape &s, const void *q, const void *K, const void *V,
+                      const int32_t *l_kv, float *out, void *ws, size_t ws_bytes,
+                      cudaStream_t st) {
+  if (!dense_supports(s.h_q, s.h_k, s.h_v)) return SAGA_ERR_UNSUPPORTED;
+  saga_status r = check_inputs(s, q, K, l_kv);
+  if (r != SAGA_OK) return r;
+  if (V == nullptr || !aligned(V, 16) || out == nullptr || !aligned(out, 16))
+    return SAGA_ERR_INVALID_ARG;
+  if ((r = check_ws(s, ws, ws_bytes)) != SAGA_OK) return r;
+  const Plan pl = make_plan(s, false);
+  StepParams p = base_params(s, pl, q, K, V, l_kv, ws);
+  cudaError_t e = launch_dense_split(p, s.dtype, s.d, st);
+  if (e != cudaSuccess) return SAGA_ERR_CUDA;
+  e = launch_combine(p.partials, l_kv, p.err, out, nullptr, s.B, s.h_q, s.d, pl.S, pl.split_len,
+                     s.cap, s.max_l_kv, st);
+  return cuda_status(e);
+}
+
 }  // namespace
 
 // Scratch a plain step needs (error word + per-split states; no score rows).
@@ -274,21 +294,16 @@ saga_status gqa_dense_decode(const saga_shape *shape, const void *q, const void 
                              size_t ws_bytes, saga_stream_t stream) {
   saga_status r = check_shape(shape);
   if (r != SAGA_OK) return r;
-  const saga_shape &s = *shape;
-  if (s.h_k != s.h_v) return SAGA_ERR_INVALID_ARG;
-  if (s.h_q / s.h_k > 8) return SAGA_ERR_UNSUPPORTED;
-  if ((r = check_inputs(s, q, K, l_kv)) != SAGA_OK) return r;
-  if (V == nullptr || !aligned(V, 16) || out == nullptr || !aligned(out, 16))
-    return SAGA_ERR_INVALID_ARG;
-  if ((r = check_ws(s, ws, ws_bytes)) != SAGA_OK) return r;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const Plan pl = make_plan(s, false);
-  StepParams p = base_params(s, pl, q, K, V, l_kv, ws);
-  cudaError_t e = launch_dense_split(p, s.dtype, s.d, group_pad(s), st);
-  if (e != cudaSuccess) return SAGA_ERR_CUDA;
-  e = launch_combine(p.partials, l_kv, p.err, out, nullptr, s.B, s.h_q, s.d, pl.S, pl.split_len,
-                     s.cap, s.max_l_kv, st);
-  return cuda_status(e);
+  if (shape->h_k != shape->h_v) return SAGA_ERR_INVALID_ARG;
+  return run_dense(*shape, q, K, V, l_kv, out, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+saga_status saga_dense_decode(const saga_shape *shape, const void *q, const void *K,
+                              const void *V, const int32_t *l_kv, float *out, void *ws,
+                              size_t ws_bytes, saga_stream_t stream) {
+  saga_status r = check_shape(shape);
+  if (r != SAGA_OK) return r;
+  return run_dense(*shape, q, K, V, l_kv, out, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 saga_status saga_debug_scores(const saga_shape *shape, const void *q, const void *K,

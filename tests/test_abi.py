@@ -107,3 +107,15 @@ def test_bad_pointers_and_workspace(lib):
     s2 = saga.shape(1, 32, 2, 8, 64, saga.SAGA_BF16, 4096)
     s2.k_stride_h = 4096 * 64 + 4
     assert saga.workspace_size(s2, 8) == 0
+
+
+@pytest.mark.parametrize("hq,hk,hv,code", [
+    (16, 2, 16, saga.SAGA_ERR_UNSUPPORTED),     # eight value heads per key head
+    (20, 2, 4, saga.SAGA_ERR_UNSUPPORTED),      # group of 10 query heads over 2 value heads
+    (32, 2, 8, saga.SAGA_ERR_WORKSPACE),        # supported: gets as far as the workspace check
+])
+def test_saga_dense_shapes(lib, hq, hk, hv, code):
+    s = saga.shape(1, hq, hk, hv, 64, saga.SAGA_BF16, 4096)
+    fake = 1 << 40   # never dereferenced: validation fails first
+    rc = lib.saga_dense_decode(ctypes.byref(s), fake, fake, fake, fake, fake, None, 0, None)
+    assert rc == code

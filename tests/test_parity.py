@@ -166,6 +166,41 @@ def test_dense_gqa_matches_oracle(name, samples):
 
 
 # ---------------------------------------------------------------------------
+# SAGA full attention (asymmetric heads, every position): the ablation arm
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("name,samples", [("tiny_f32", [(0, 0), (0, 3)]),
+                                          ("llama1b_32k", [(0, 0), (0, 13), (0, 31)]),
+                                          ("qwen1p5b_128k", [(0, 2), (0, 11)]),
+                                          ("llama1b_stack16_b8_128k", [(5, 6), (7, 29)])])
+def test_saga_full_matches_oracle(name, samples):
+    w = synth.WORKLOADS[name]
+    lens = synth.seq_lens(w)
+    K = dev_cache(w, 0, "K", w.h_k, w.l_kv)
+    V = dev_cache(w, 0, "V", w.h_v, w.l_kv)
+    shp = saga_shape(w)
+    ws = saga.Workspace(shp)
+    qs = synth.queries(w, 0, 1)
+    out = torch.zeros(w.B, w.h_q, w.d, dtype=torch.float32, device="cuda")
+    l = torch.from_numpy(lens).cuda()
+    saga.dense_decode(shp, to_dev(qs[0]), K, V, l, out, ws)
+    torch.cuda.synchronize()
+    assert saga.read_device_error(ws) == 0
+    o = out.cpu().numpy()
+    q64 = synth.widen(qs[0])
+    for (b, j) in samples:
+        L = int(lens[b])
+        kh = orc.key_head(j, w.h_q, w.h_k)
+        vh = orc.value_head(j, w.h_q, w.h_v)
+        Kr = synth.widen(synth.cache_rows(w, 0, "K", b, kh, 0, L))
+        Vr = synth.widen(synth.cache_rows(w, 0, "V", b, vh, 0, L))
+        A = Kr @ q64[b, j] / np.sqrt(w.d)
+        ref = orc.sparse_attend(A, Vr, np.arange(L))
+        assert rel_err(o[b, j].astype(np.float64), ref) <= OUT_TOL[w.dtype]
+    del K, V
+    torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------------------
 # edge cases on small host-generated inputs
 # ---------------------------------------------------------------------------
 def small_case(dtype, B, h_q, h_k, h_v, d, cap, seed):
