@@ -26,6 +26,10 @@ Readings where the pages are silent (each also listed in the design notes):
   * An empty selection gives an output row of zeros.
   * Refresh steps are t = 0, R, 2R, ...; the refreshed tau applies to the
     same step's selection.
+  * Exact top-N attention (Eq. 6) keeps exactly min(N, l_kv) positions; among
+    equal scores the lower position wins (the pages fix no tie-break).
+  * Decoding appends the token's key and value rows at position l_kv[b] of
+    every head and grows l_kv[b] by one before the step attends.
 
 Everything is computed in float64 from the exact values of the stored inputs,
 with no blocking, fusion or reordering beyond the definitions above.
@@ -188,3 +192,49 @@ def nth_largest_f32(row_f32, N):
         return np.float32(NEG_INF)
     keys = np.sort(f32_order_key(row_f32))[::-1]
     return f32_from_order_key(keys[N - 1:N])[0]
+
+
+# --------------------------------------------------------------------------
+# exact top-N attention (Eq. 6), ties broken towards the lower position
+# --------------------------------------------------------------------------
+def top_n_exact(row, N):
+    """Positions of the min(N, len(row)) largest entries of `row`; among equal
+    entries the lower position is taken first."""
+    row = np.asarray(row, dtype=np.float64)
+    order = np.lexsort((np.arange(row.size), -row))   # by -value, then position
+    return np.sort(order[:min(N, row.size)])
+
+
+def topn_step(q, K, V, l_kv, N):
+    """One exact top-N attention step (Eq. 6 + Eq. 7) for every (b, j)."""
+    B, h_q, d = q.shape
+    h_v = V.shape[1]
+    A = scores(q, K, l_kv)
+    sels, out = [], np.zeros((B, h_q, d))
+    for b in range(B):
+        row_sels = []
+        for j in range(h_q):
+            idx = top_n_exact(A[b][j], N)
+            out[b, j] = sparse_attend(A[b][j], V[b, value_head(j, h_q, h_v)], idx)
+            row_sels.append(idx)
+        sels.append(row_sels)
+    return sels, out
+
+
+# --------------------------------------------------------------------------
+# KV-cache append (the decode step's input side)
+# --------------------------------------------------------------------------
+def append(K, V, l_kv, k_new, v_new):
+    """Write each sequence's new key rows k_new [B][h_k][d] and value rows
+    v_new [B][h_v][d] at position l_kv[b] of every head; returns copies of
+    K, V and l_kv + 1."""
+    K, V = np.array(K, copy=True), np.array(V, copy=True)
+    l_kv = np.array(l_kv, copy=True)
+    for b in range(K.shape[0]):
+        t = int(l_kv[b])
+        if t >= K.shape[2]:
+            raise ValueError("cache full")
+        K[b, :, t, :] = k_new[b]
+        V[b, :, t, :] = v_new[b]
+        l_kv[b] = t + 1
+    return K, V, l_kv

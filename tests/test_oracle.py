@@ -232,3 +232,90 @@ def test_chain_refreshes_on_schedule():
         np.testing.assert_array_equal(taus[t], orc.refresh(qs[r], K, l, 9))
         s, o = orc.decode_step(qs[t], K, V, l, taus[t])
         np.testing.assert_array_equal(outs[t], o)
+
+
+# ---------------------------------------------------------------------------
+# exact top-N (Eq. 6) with ties broken towards the lower position
+# ---------------------------------------------------------------------------
+def test_top_n_exact_brute_force_with_ties():
+    rng = np.random.default_rng(11)
+    for trial in range(300):
+        L = int(rng.integers(1, 40))
+        row = rng.integers(-3, 4, size=L).astype(np.float64)   # many ties
+        N = int(rng.integers(1, 50))
+        ranked = sorted(range(L), key=lambda t: (-row[t], t))
+        want = sorted(ranked[:min(N, L)])
+        assert list(orc.top_n_exact(row, N)) == want
+
+
+def test_top_n_exact_keeps_exactly_n():
+    rng = np.random.default_rng(12)
+    for trial in range(50):
+        L = int(rng.integers(1, 200))
+        row = np.round(rng.standard_normal(L), 1)            # ties at every threshold
+        N = int(rng.integers(1, 250))
+        assert orc.top_n_exact(row, N).size == min(N, L)
+
+
+def test_top_n_exact_without_ties_is_the_refresh_selection():
+    rng = np.random.default_rng(13)
+    for trial in range(50):
+        L = int(rng.integers(2, 500))
+        row = rng.standard_normal(L)
+        N = int(rng.integers(1, L))
+        tau = orc.nth_largest(row, N)
+        assert np.array_equal(orc.top_n_exact(row, N), orc.select(row, tau))
+
+
+def test_topn_step_matches_atop_n_refresh_without_ties():
+    rng = np.random.default_rng(14)
+    B, h_q, h_k, h_v, d, L, N = 2, 8, 2, 4, 16, 90, 11
+    q = rng.standard_normal((B, h_q, d))
+    K = rng.standard_normal((B, h_k, L, d))
+    V = rng.standard_normal((B, h_v, L, d))
+    l = np.array([L, 57])
+    sel_t, out_t = orc.topn_step(q, K, V, l, N)
+    tau = orc.refresh(q, K, l, N)
+    sel_a, out_a = orc.decode_step(q, K, V, l, tau)
+    np.testing.assert_allclose(out_t, out_a, rtol=0, atol=1e-12)
+    for b in range(B):
+        for j in range(h_q):
+            assert np.array_equal(sel_t[b][j], sel_a[b][j])
+
+
+# ---------------------------------------------------------------------------
+# KV-cache append and the growing-context decode loop
+# ---------------------------------------------------------------------------
+def test_append_then_attend_equals_concatenated_cache():
+    rng = np.random.default_rng(15)
+    B, h_q, h_k, h_v, d, cap = 2, 8, 2, 4, 16, 64
+    l0 = np.array([20, 33])
+    K = rng.standard_normal((B, h_k, cap, d))
+    V = rng.standard_normal((B, h_v, cap, d))
+    K2, V2, l = K, V, l0.copy()
+    steps = 5
+    kn = rng.standard_normal((steps, B, h_k, d))
+    vn = rng.standard_normal((steps, B, h_v, d))
+    for s_ in range(steps):
+        K2, V2, l = orc.append(K2, V2, l, kn[s_], vn[s_])
+    assert np.array_equal(l, l0 + steps)
+    q = rng.standard_normal((B, h_q, d))
+    got = orc.dense_attend(q, K2, V2, l)
+    for b in range(B):
+        Kc = np.concatenate([K[b, :, :l0[b]], np.transpose(kn[:, b], (1, 0, 2))], axis=1)
+        Vc = np.concatenate([V[b, :, :l0[b]], np.transpose(vn[:, b], (1, 0, 2))], axis=1)
+        for j in range(h_q):
+            kh, vh = orc.key_head(j, h_q, h_k), orc.value_head(j, h_q, h_v)
+            A = Kc[kh] @ q[b, j] / np.sqrt(d)
+            w = np.exp(A - A.max())
+            np.testing.assert_allclose(got[b, j], (w @ Vc[vh]) / w.sum(), rtol=1e-12, atol=1e-12)
+    # positions before the append point and after it stay as they were
+    for b in range(B):
+        assert np.array_equal(K2[b, :, :l0[b]], K[b, :, :l0[b]])
+        assert np.array_equal(K2[b, :, l0[b] + steps:], K[b, :, l0[b] + steps:])
+
+
+def test_append_refuses_a_full_cache():
+    K = np.zeros((1, 1, 4, 2)); V = np.zeros((1, 1, 4, 2))
+    with pytest.raises(ValueError):
+        orc.append(K, V, np.array([4]), np.ones((1, 1, 2)), np.ones((1, 1, 2)))
