@@ -151,6 +151,26 @@ saga_status saga_refresh_threshold(const saga_shape *shape, const void *q,
                                    saga_stream_t stream);
 
 /*
+ * Exact top-N attention for this step (Top-N Attention, Eq. 6, then Eq. 7):
+ * for every (b, j) the min(N, l_kv[b]) positions with the largest scores are
+ * kept, ties broken towards the lower position (the paper fixes no
+ * tie-break; scores are ordered by IEEE totalOrder, so -0 < +0), and
+ * out[b][j] is the softmax-weighted sum of their value rows. It computes
+ * the scores, selects the N-th largest (as a refresh does), finds the last
+ * tied position taken, and runs the step with that rule; nothing persists
+ * between calls (an R = 1 reference for Atop-N).
+ *   Arguments as for saga_refresh_threshold without tau (kept in the
+ *   workspace); V and out are required; scores, sel_count and sel_mask are
+ *   nullable outputs with the same layouts. sel_count[b][j] is exactly
+ *   min(N, l_kv[b]).
+ */
+saga_status saga_topn_step(const saga_shape *shape, const void *q,
+                           const void *K, const void *V, const int32_t *l_kv,
+                           int32_t N, float *out, int32_t *sel_count,
+                           uint8_t *sel_mask, float *scores, void *ws,
+                           size_t ws_bytes, saga_stream_t stream);
+
+/*
  * Full-attention GQA decode (Eq. 2-4 over every t < l_kv[b]): the dense
  * baseline the sparse step is measured against. Requires h_k == h_v and
  * h_q / h_k <= 16 (else SAGA_ERR_INVALID_ARG / SAGA_ERR_UNSUPPORTED).
@@ -176,6 +196,27 @@ saga_status saga_dense_decode(const saga_shape *shape, const void *q,
                               const void *K, const void *V,
                               const int32_t *l_kv, float *out, void *ws,
                               size_t ws_bytes, saga_stream_t stream);
+
+/*
+ * KV-cache append, the input side of a decode step (Background on
+ * autoregressive decoding: each generated token's key and value join the
+ * cache before the next attention): for every sequence b, the new key rows
+ * k_new[b][0..h_k-1][0..d-1] and value rows v_new[b][0..h_v-1][0..d-1]
+ * (contiguous, the cache dtype) are written at position l_kv[b] of every
+ * head of K and V, then l_kv[b] grows by one, all on the device and in
+ * stream order, so a following step or refresh attends over l_kv[b] + 1
+ * positions.
+ *   K, V      the caches described by `shape`, written at one position per head.
+ *   l_kv      [B] int32, read and incremented on the device.
+ *   ws        a workspace (only its error word is used; >= 256 bytes).
+ * A sequence whose l_kv[b] is already >= cap (or negative) is left as it is
+ * and the workspace's error word receives SAGA_DEVERR_LKV_TOO_LONG (or
+ * _NEGATIVE). Steps plan with shape->max_l_kv, so callers that grow the
+ * context set max_l_kv to the longest length they will reach.
+ */
+saga_status saga_append_kv(const saga_shape *shape, const void *k_new,
+                           const void *v_new, void *K, void *V, int32_t *l_kv,
+                           void *ws, size_t ws_bytes, saga_stream_t stream);
 
 /*
  * saga_decode_step without a workspace argument, for callers that cannot

@@ -56,6 +56,9 @@ _SIGS = {
                                               _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "gqa_dense_decode": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "saga_dense_decode": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "saga_append_kv": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "saga_topn_step": (ctypes.c_int, [_SP, _P, _P, _P, _P, ctypes.c_int32, _P, _P, _P, _P, _P,
+                                      ctypes.c_size_t, _P]),
     "saga_debug_scores": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "saga_decode_step_noalloc": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P, _P, _P]),
     "saga_read_device_error": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_int32)]),
@@ -169,6 +172,22 @@ def dense_decode(shp, q, K, V, l_kv, out, ws, stream=None):
     p, n = _ws(ws)
     _check(load().saga_dense_decode(ctypes.byref(shp), _ptr(q), _ptr(K), _ptr(V), _ptr(l_kv),
                                     _ptr(out), p, n, _stream(stream)), "saga_dense_decode")
+
+
+def topn_step(shp, q, K, V, l_kv, N, out, ws, sel_count=None, sel_mask=None, scores=None,
+              stream=None):
+    """Exact top-N attention (ties to the lower position) for this step."""
+    p, n = _ws(ws)
+    _check(load().saga_topn_step(ctypes.byref(shp), _ptr(q), _ptr(K), _ptr(V), _ptr(l_kv), N,
+                                 _ptr(out), _ptr(sel_count), _ptr(sel_mask), _ptr(scores), p, n,
+                                 _stream(stream)), "saga_topn_step")
+
+
+def append_kv(shp, k_new, v_new, K, V, l_kv, ws, stream=None):
+    """Write the token's key/value rows at position l_kv[b] and grow l_kv."""
+    p, n = _ws(ws)
+    _check(load().saga_append_kv(ctypes.byref(shp), _ptr(k_new), _ptr(v_new), _ptr(K), _ptr(V),
+                                 _ptr(l_kv), p, n, _stream(stream)), "saga_append_kv")
 
 
 NOALLOC_SCRATCH_BYTES = 4 << 20

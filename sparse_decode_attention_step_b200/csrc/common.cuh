@@ -18,6 +18,7 @@ struct StepParams {
   const void *V;
   const int32_t *l_kv;
   const float *tau;
+  const int32_t *tie;       // nullable [B][h_q]: exact top-N, keep A == tau only at t <= tie
   const float *scores_in;   // from-scores mode: [B][h_q][row_stride]
   float *scores_out;        // dump mode: [B][h_q][row_stride]
   float *partials;          // [B][h_q][S][d + kRecPad]

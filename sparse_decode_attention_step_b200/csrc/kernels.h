@@ -8,7 +8,9 @@
 
 namespace saga {
 
-enum { kModeDump = 0, kModeStep = 1, kModeFromScores = 2 };
+// kModeStepTies: a step that keeps A > tau, and A == tau only at positions
+// t <= tie[b][j] (exact top-N with ties broken towards the lower position).
+enum { kModeDump = 0, kModeStep = 1, kModeFromScores = 2, kModeStepTies = 3 };
 
 // Split kernel over grid (S, B * h_k); gp = h_q / h_k rounded up to 4.
 cudaError_t launch_saga_split(const StepParams &p, int mode, int dtype, int d, int gp,
@@ -31,14 +33,24 @@ cudaError_t launch_combine(const float *partials, const int32_t *l_kv, int32_t *
 // tau[b][j] = N-th largest of the stored score row (b, j), or -inf if N >= l_kv[b].
 // hist0: nullable [B][h_q][256] top-byte histograms of the rows' order keys
 // (from the score pass); without it the kernel makes one more pass.
+// tie: nullable [B][h_q]; receives the position of the last entry equal to
+// tau that the N largest take when ties go to the lower position (one more
+// pass over the row), or INT32_MAX when N >= l_kv[b].
 cudaError_t launch_radix_select(const float *scores, int64_t row_stride, const int32_t *l_kv,
                                 int N, float *tau, int B, int h_q, int64_t cap, int64_t max_l_kv,
-                                const uint32_t *hist0, cudaStream_t st);
+                                const uint32_t *hist0, int32_t *tie, cudaStream_t st);
 
 // Dense (full-attention) split kernel over grid (S, B * h_k): GQA (h_k == h_v,
 // h_q / h_k <= 16) or SAGA heads (h_v / h_k in {2, 4}, h_q / h_k in {4, 8, 12, 16}).
 bool dense_supports(int h_q, int h_k, int h_v);
 cudaError_t launch_dense_split(const StepParams &p, int dtype, int d, cudaStream_t st);
+
+// KV-cache append over grid (B): rows k_new [B][h_k][d] and v_new [B][h_v][d]
+// (contiguous) to position l_kv[b], then l_kv[b] += 1. Strides in elements.
+cudaError_t launch_append(const void *k_new, const void *v_new, void *K, void *V, int32_t *l_kv,
+                          int32_t *err, int B, int h_k, int h_v, int d, int esz, int64_t k_sb,
+                          int64_t k_sh, int64_t v_sb, int64_t v_sh, int64_t cap,
+                          cudaStream_t st);
 
 // Plain step with a caller-chosen scratch buffer (see saga_decode_step_noalloc).
 size_t plain_step_scratch_bytes(const saga_shape &s);

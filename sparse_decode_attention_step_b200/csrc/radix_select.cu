@@ -15,6 +15,12 @@
 // share one binade), a third pass copies only the keys that match the first
 // two digits; only if even those do not fit, digits 2 and 3 take one pass
 // over the row each.
+//
+// Exact top-N (Eq. 6 with ties to the lower position) also needs, when tau is
+// tied, how far along the row the taken ties reach: after the last digit the
+// rank left inside tau's bucket is the number k of entries equal to tau that
+// the N largest include, and one more pass in position order finds the
+// position of the k-th of them.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -28,6 +34,8 @@ constexpr int kCand = 32768;                        // candidate keys kept on ch
 struct Shared {
   uint32_t hist[256];
   uint32_t digit, rem, n_cand;
+  uint32_t wsum[32];
+  int32_t found;
 };
 
 // Histogram of digit `shift` over keys with (k & mask) == prefix, one shared
@@ -105,7 +113,8 @@ __device__ __forceinline__ void for_row(const float *row, int64_t L, int tid, F 
 __global__ void __launch_bounds__(kThreads, 1)
 radix_select_kernel(const float *__restrict__ scores, int64_t row_stride,
                     const int32_t *__restrict__ l_kv, int N, float *__restrict__ tau, int h_q,
-                    int64_t cap, int64_t max_l_kv, const uint32_t *__restrict__ hist0) {
+                    int64_t cap, int64_t max_l_kv, const uint32_t *__restrict__ hist0,
+                    int32_t *__restrict__ tie) {
   __shared__ Shared sh;
   extern __shared__ uint32_t cand[];
   const int bj = blockIdx.x;
@@ -116,7 +125,10 @@ radix_select_kernel(const float *__restrict__ scores, int64_t row_stride,
   if (L < 0) L = 0;
   if (L > hi) L = hi;
   if (static_cast<int64_t>(N) >= L) {
-    if (tid == 0) tau[bj] = -INFINITY;
+    if (tid == 0) {
+      tau[bj] = -INFINITY;
+      if (tie != nullptr) tie[bj] = INT32_MAX;
+    }
     return;
   }
   const float *row = scores + static_cast<int64_t>(bj) * row_stride;
@@ -211,13 +223,58 @@ radix_select_kernel(const float *__restrict__ scores, int64_t row_stride,
     __syncthreads();
   }
   if (tid == 0) tau[bj] = from_order_key(prefix);
+  if (tie == nullptr) return;
+
+  // ---- position of the k-th entry equal to tau, in position order -------
+  const uint32_t k = sh.rem;                    // 1 <= k <= #(entries equal to tau)
+  if (tid == 0) sh.found = -1;
+  __syncthreads();
+  uint32_t before = 0;                          // matches in earlier chunks
+  constexpr int64_t kSpan = static_cast<int64_t>(kThreads) * 4;
+  for (int64_t t0 = 0; t0 < L; t0 += kSpan) {
+    const int64_t i = t0 + static_cast<int64_t>(tid) * 4;
+    uint32_t hits = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (i + e < L && order_key(row[i + e]) == prefix) hits |= 1u << e;
+    const uint32_t c = __popc(hits);
+    // exclusive prefix of c over the CTA, in thread (= position) order
+    uint32_t incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) sh.wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      uint32_t ws = sh.wsum[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, ws, o);
+        if (lane >= o) ws += y;
+      }
+      sh.wsum[lane] = ws;                       // inclusive over warps
+    }
+    __syncthreads();
+    const uint32_t excl = before + (warp > 0 ? sh.wsum[warp - 1] : 0u) + (incl - c);
+    if (c > 0 && excl < k && k <= excl + c) {
+      uint32_t need = k - excl, hh = hits;
+      while (--need) hh &= hh - 1u;
+      sh.found = static_cast<int32_t>(i + __ffs(hh) - 1);
+    }
+    before += sh.wsum[kThreads / 32 - 1];
+    __syncthreads();
+    if (sh.found >= 0) break;
+  }
+  if (tid == 0) tie[bj] = sh.found;
 }
 
 }  // namespace
 
 cudaError_t launch_radix_select(const float *scores, int64_t row_stride, const int32_t *l_kv,
                                 int N, float *tau, int B, int h_q, int64_t cap, int64_t max_l_kv,
-                                const uint32_t *hist0, cudaStream_t st) {
+                                const uint32_t *hist0, int32_t *tie, cudaStream_t st) {
   static bool attr_set = false;
   const int smem = kCand * static_cast<int>(sizeof(uint32_t));
   if (!attr_set) {
@@ -227,7 +284,7 @@ cudaError_t launch_radix_select(const float *scores, int64_t row_stride, const i
     attr_set = true;
   }
   radix_select_kernel<<<B * h_q, kThreads, smem, st>>>(scores, row_stride, l_kv, N, tau, h_q,
-                                                       cap, max_l_kv, hist0);
+                                                       cap, max_l_kv, hist0, tie);
   return cudaGetLastError();
 }
 

@@ -24,7 +24,7 @@ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 struct Plan {
   int S;                    // splits per (b, key head)
   int64_t split_len;        // positions per split
-  size_t off_partials, off_scores, off_hist, total;
+  size_t off_partials, off_scores, off_hist, off_tau, off_tie, total;
 };
 
 bool use_tc(const saga_shape &s);
@@ -54,7 +54,9 @@ Plan make_plan(const saga_shape &s, bool persistent) {
   p.off_partials = kAlign;   // [0, 256): device error word
   p.off_scores = align_up(p.off_partials + static_cast<size_t>(s.B) * s.h_q * p.S * rec);
   p.off_hist = align_up(p.off_scores + static_cast<size_t>(s.B) * s.h_q * s.max_l_kv * sizeof(float));
-  p.total = align_up(p.off_hist + static_cast<size_t>(s.B) * s.h_q * 256 * sizeof(uint32_t));
+  p.off_tau = align_up(p.off_hist + static_cast<size_t>(s.B) * s.h_q * 256 * sizeof(uint32_t));
+  p.off_tie = align_up(p.off_tau + static_cast<size_t>(s.B) * s.h_q * sizeof(float));
+  p.total = align_up(p.off_tie + static_cast<size_t>(s.B) * s.h_q * sizeof(int32_t));
   return p;
 }
 
@@ -274,7 +276,7 @@ saga_status saga_refresh_threshold(const saga_shape *shape, const void *q, const
   if (e != cudaSuccess) return SAGA_ERR_CUDA;
   // 2. exact N-th largest per row
   e = launch_radix_select(rows, s.max_l_kv, l_kv, N, tau, s.B, s.h_q, s.cap, s.max_l_kv, hist,
-                          st);
+                          nullptr, st);
   if (e != cudaSuccess) return SAGA_ERR_CUDA;
   if (V == nullptr) return SAGA_OK;
   // 3. this step's select + PV with the fresh tau. Tensor-core shapes: the
@@ -285,6 +287,54 @@ saga_status saga_refresh_threshold(const saga_shape *shape, const void *q, const
   p.tau = tau;
   p.sel_mask = sel_mask;
   if (use_tc(s)) return run_step(s, pl, p, kModeStep, out, sel_count, st);
+  p.scores_in = rows;
+  return run_step(s, pl, p, kModeFromScores, out, sel_count, st);
+}
+
+saga_status saga_topn_step(const saga_shape *shape, const void *q, const void *K,
+                           const void *V, const int32_t *l_kv, int32_t N, float *out,
+                           int32_t *sel_count, uint8_t *sel_mask, float *scores, void *ws,
+                           size_t ws_bytes, saga_stream_t stream) {
+  saga_status r = check_shape(shape);
+  if (r != SAGA_OK) return r;
+  const saga_shape &s = *shape;
+  if ((r = check_inputs(s, q, K, l_kv)) != SAGA_OK) return r;
+  if (N < 1 || V == nullptr || out == nullptr || !aligned(V, 16) || !aligned(out, 16))
+    return SAGA_ERR_INVALID_ARG;
+  if ((scores && !aligned(scores, 4)) || (sel_count && !aligned(sel_count, 4)))
+    return SAGA_ERR_INVALID_ARG;
+  if ((r = check_ws(s, ws, ws_bytes)) != SAGA_OK) return r;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const Plan pl = saga_plan(s);
+  StepParams p = base_params(s, pl, q, K, V, l_kv, ws);
+  char *wsb = static_cast<char *>(ws);
+  float *rows = scores != nullptr ? scores : reinterpret_cast<float *>(wsb + pl.off_scores);
+  float *tau = reinterpret_cast<float *>(wsb + pl.off_tau);
+  int32_t *tie = reinterpret_cast<int32_t *>(wsb + pl.off_tie);
+  // 1. score rows (tensor-core kernel: with the top-byte histogram of every row)
+  uint32_t *hist = nullptr;
+  if (use_tc(s)) {
+    hist = reinterpret_cast<uint32_t *>(wsb + pl.off_hist);
+    if (cudaMemsetAsync(hist, 0, static_cast<size_t>(s.B) * s.h_q * 256 * sizeof(uint32_t), st) !=
+        cudaSuccess)
+      return SAGA_ERR_CUDA;
+  }
+  p.scores_out = rows;
+  p.hist = hist;
+  cudaError_t e = launch_split(s, p, kModeDump, st);
+  if (e != cudaSuccess) return SAGA_ERR_CUDA;
+  // 2. the N-th largest and, when it is tied, the last tied position taken
+  e = launch_radix_select(rows, s.max_l_kv, l_kv, N, tau, s.B, s.h_q, s.cap, s.max_l_kv, hist,
+                          tie, st);
+  if (e != cudaSuccess) return SAGA_ERR_CUDA;
+  // 3. the step over exactly those positions (bit-identical scores again on
+  // the tensor-core path, the stored rows otherwise)
+  p.scores_out = nullptr;
+  p.hist = nullptr;
+  p.tau = tau;
+  p.tie = tie;
+  p.sel_mask = sel_mask;
+  if (use_tc(s)) return run_step(s, pl, p, kModeStepTies, out, sel_count, st);
   p.scores_in = rows;
   return run_step(s, pl, p, kModeFromScores, out, sel_count, st);
 }
@@ -304,6 +354,24 @@ saga_status saga_dense_decode(const saga_shape *shape, const void *q, const void
   saga_status r = check_shape(shape);
   if (r != SAGA_OK) return r;
   return run_dense(*shape, q, K, V, l_kv, out, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+saga_status saga_append_kv(const saga_shape *shape, const void *k_new, const void *v_new,
+                           void *K, void *V, int32_t *l_kv, void *ws, size_t ws_bytes,
+                           saga_stream_t stream) {
+  saga_status r = check_shape(shape);
+  if (r != SAGA_OK) return r;
+  const saga_shape &s = *shape;
+  if (k_new == nullptr || v_new == nullptr || K == nullptr || V == nullptr || l_kv == nullptr)
+    return SAGA_ERR_INVALID_ARG;
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(K, 16) || !aligned(V, 16) ||
+      !aligned(l_kv, 4))
+    return SAGA_ERR_INVALID_ARG;
+  if (ws == nullptr || !aligned(ws, kAlign) || ws_bytes < kAlign) return SAGA_ERR_WORKSPACE;
+  const int esz = s.dtype == SAGA_F32 ? 4 : 2;
+  return cuda_status(launch_append(k_new, v_new, K, V, l_kv, static_cast<int32_t *>(ws), s.B, s.h_k,
+                                   s.h_v, s.d, esz, s.k_stride_b, s.k_stride_h, s.v_stride_b,
+                                   s.v_stride_h, s.cap, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 saga_status saga_debug_scores(const saga_shape *shape, const void *q, const void *K,

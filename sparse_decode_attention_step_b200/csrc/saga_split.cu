@@ -91,6 +91,7 @@ saga_split_kernel(const StepParams p, const int mode) {
 
   __shared__ __align__(16) float qs[D * GP];
   __shared__ float tau_s[GP];
+  __shared__ int32_t tie_s[GP];
   __shared__ int sel_t[GP][kChunk];
   __shared__ float sel_a[GP][kChunk];
   __shared__ int warp_off[kWarps][GP];
@@ -111,7 +112,10 @@ saga_split_kernel(const StepParams p, const int mode) {
     int i = idx / GP, g = idx % GP;
     qs[idx] = g < G ? widen1(qg + (j0 + g) * p.q_sh + i) : 0.f;
   }
-  if (tid < GP) tau_s[tid] = (tid < G && mode != kModeDump) ? p.tau[b * p.h_q + j0 + tid] : 0.f;
+  if (tid < GP) {
+    tau_s[tid] = (tid < G && mode != kModeDump) ? p.tau[b * p.h_q + j0 + tid] : 0.f;
+    tie_s[tid] = (tid < G && p.tie != nullptr) ? p.tie[b * p.h_q + j0 + tid] : -1;
+  }
   __syncthreads();
 
   const T *krow0 = static_cast<const T *>(p.K) + b * p.k_sb + kh * p.k_sh;
@@ -156,7 +160,14 @@ saga_split_kernel(const StepParams p, const int mode) {
     const uint32_t lt_mask = (1u << lane) - 1u;
 #pragma unroll
     for (int g = 0; g < GP; ++g) {
-      const bool sel = valid && g < G && A[g] >= tau_s[g];
+      bool sel;
+      if (p.tie != nullptr) {
+        // exact top-N: totalOrder above tau, or equal up to the tie position
+        const uint32_t kx = order_key(A[g]), kt = order_key(tau_s[g]);
+        sel = valid && g < G && (kx > kt || (kx == kt && t <= tie_s[g]));
+      } else {
+        sel = valid && g < G && A[g] >= tau_s[g];
+      }
       const uint32_t bal = __ballot_sync(0xffffffffu, sel);
       if (lane == 0) warp_off[warp][g] = __popc(bal);
       pos[g] = __popc(bal & lt_mask);

@@ -79,6 +79,7 @@ struct Header {
   uint32_t tmem_base;
   int abort;
   alignas(16) float tau[kN];
+  int32_t tie[kN];           // tie mode: last position at which A == tau is kept
 };
 
 template <int D>
@@ -450,9 +451,11 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
       if (!unit_at(p, u, false, un)) continue;
       const int j0 = un.kh * G;
       const int64_t row0 = static_cast<int64_t>(un.b * p.h_q + j0) * p.row_stride;
-      if (MODE == kModeStep) {
-        if (widx == 0 && lane < kN)
+      if (MODE != kModeDump) {
+        if (widx == 0 && lane < kN) {
           h->tau[lane] = lane < G ? p.tau[un.b * p.h_q + j0 + lane] : INFINITY;
+          if (MODE == kModeStepTies) h->tie[lane] = lane < G ? p.tie[un.b * p.h_q + j0 + lane] : -1;
+        }
         workers_sync<D>();
       }
 #pragma unroll
@@ -521,7 +524,15 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
             for (int e = 0; e < 4; ++e) {
               const int a = 4 * a4 + e;
               const float x = A[a] * p.scale;
-              const bool keep = valid && x >= tt[e];
+              bool keep;
+              if constexpr (MODE == kModeStepTies) {
+                // totalOrder, as the threshold was selected: above tau, or
+                // equal to it up to the last position the top N take
+                const uint32_t kx = order_key(x), kt = order_key(tt[e]);
+                keep = valid && (kx > kt || (kx == kt && t <= h->tie[a]));
+              } else {
+                keep = valid && x >= tt[e];
+              }
               sel |= static_cast<uint32_t>(keep) << a;
               A[a] = keep ? x : -INFINITY;
             }
@@ -709,7 +720,7 @@ bool saga_tc_supports(int dtype, int d, int h_q, int h_k, int h_v) {
 cudaError_t launch_saga_tc(const StepParams &p, int mode, int d, cudaStream_t st) {
   HeadMap hm;
   if (!make_head_map(p.h_q, p.h_k, p.h_v, hm)) return cudaErrorInvalidValue;
-  if (mode != kModeDump && mode != kModeStep) return cudaErrorInvalidValue;
+  if (mode != kModeDump && mode != kModeStep && mode != kModeStepTies) return cudaErrorInvalidValue;
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return cudaErrorNotSupported;
   int dev = 0;
@@ -741,12 +752,16 @@ cudaError_t launch_saga_tc(const StepParams &p, int mode, int d, cudaStream_t st
             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  if (d == 64)
-    return mode == kModeDump ? launch_tc<64, kModeDump>(p, kmap, qmap, hm, dev, st)
-                             : launch_tc<64, kModeStep>(p, kmap, qmap, hm, dev, st);
-  if (d == 128)
-    return mode == kModeDump ? launch_tc<128, kModeDump>(p, kmap, qmap, hm, dev, st)
-                             : launch_tc<128, kModeStep>(p, kmap, qmap, hm, dev, st);
+  if (d == 64) {
+    if (mode == kModeDump) return launch_tc<64, kModeDump>(p, kmap, qmap, hm, dev, st);
+    if (mode == kModeStep) return launch_tc<64, kModeStep>(p, kmap, qmap, hm, dev, st);
+    return launch_tc<64, kModeStepTies>(p, kmap, qmap, hm, dev, st);
+  }
+  if (d == 128) {
+    if (mode == kModeDump) return launch_tc<128, kModeDump>(p, kmap, qmap, hm, dev, st);
+    if (mode == kModeStep) return launch_tc<128, kModeStep>(p, kmap, qmap, hm, dev, st);
+    return launch_tc<128, kModeStepTies>(p, kmap, qmap, hm, dev, st);
+  }
   return cudaErrorInvalidValue;
 }
 

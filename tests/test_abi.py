@@ -119,3 +119,15 @@ def test_saga_dense_shapes(lib, hq, hk, hv, code):
     fake = 1 << 40   # never dereferenced: validation fails first
     rc = lib.saga_dense_decode(ctypes.byref(s), fake, fake, fake, fake, fake, None, 0, None)
     assert rc == code
+
+
+def test_append_kv_host_checks(lib):
+    s = saga.shape(2, 16, 2, 4, 64, saga.SAGA_BF16, 4096)
+    ok = 1 << 40    # never dereferenced: validation fails first
+    call = lambda **o: lib.saga_append_kv(ctypes.byref(s), o.get("kn", ok), o.get("vn", ok),
+                                          o.get("K", ok), o.get("V", ok), o.get("l", ok),
+                                          o.get("ws", ok), o.get("n", 256), None)
+    assert call(kn=None) == saga.SAGA_ERR_INVALID_ARG
+    assert call(V=ok + 8) == saga.SAGA_ERR_INVALID_ARG        # not 16-byte aligned
+    assert call(ws=None) == saga.SAGA_ERR_WORKSPACE
+    assert call(n=255) == saga.SAGA_ERR_WORKSPACE             # room for the error word only
