@@ -46,6 +46,50 @@ __device__ __forceinline__ void dense_scores(const T *krow, const float *qs, flo
   for (int g = 0; g < GP; ++g) A[g] = acc[g] * scale;
 }
 
+// bf16 caches: the scores of one warp's 32 positions (two m16 row tiles)
+// against the GP query heads on the tensor cores (mma.sync m16n8k16, bf16 in,
+// fp32 accumulate; bf16 products are exact in fp32, so only the summation
+// order differs from the FMA chain). Rows past `last` re-read row `last`.
+// qb: the heads' B fragments, per 16-column slice and 8-head tile.
+template <int D, int NT>
+__device__ __forceinline__ void mma_scores(const uint16_t *krow0, int64_t key0, int64_t last,
+                                           const uint32_t (&qb)[D / 16][NT][2], float *sc,
+                                           int gp, int lane) {
+  const int g = lane >> 2, tq = lane & 3;
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt) {
+    const int64_t r0 = min(key0 + mt * 16 + g, last), r1 = min(key0 + mt * 16 + g + 8, last);
+    const uint32_t *p0 = reinterpret_cast<const uint32_t *>(krow0 + r0 * D);
+    const uint32_t *p1 = reinterpret_cast<const uint32_t *>(krow0 + r1 * D);
+    float d[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) d[nt][0] = d[nt][1] = d[nt][2] = d[nt][3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      const uint32_t a0 = __ldg(p0 + ks * 8 + tq), a1 = __ldg(p1 + ks * 8 + tq);
+      const uint32_t a2 = __ldg(p0 + ks * 8 + 4 + tq), a3 = __ldg(p1 + ks * 8 + 4 + tq);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+            "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+            : "+f"(d[nt][0]), "+f"(d[nt][1]), "+f"(d[nt][2]), "+f"(d[nt][3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(qb[ks][nt][0]), "r"(qb[ks][nt][1]));
+    }
+    const int row = mt * 16 + g;            // within the warp's 32 positions
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int hd = nt * 8 + tq * 2 + i;
+        if (hd < gp) {
+          sc[row * gp + hd] = d[nt][i];
+          sc[(row + 8) * gp + hd] = d[nt][2 + i];
+        }
+      }
+  }
+}
+
 __device__ __forceinline__ float widen1(const float *p) { return *p; }
 __device__ __forceinline__ float widen1(const uint16_t *p) {
   return __uint_as_float(static_cast<uint32_t>(*p) << 16);
@@ -76,7 +120,9 @@ template <typename T, int D, int GP, int VPG>
 __global__ void __launch_bounds__(kThreads) dense_split_kernel(const StepParams p) {
   constexpr int VPL = D / 32;
   constexpr int HPV = GP / VPG;              // query heads per value head (VPG > 1: GP == G)
-  __shared__ __align__(16) float qs[D * GP];
+  constexpr bool kMma = sizeof(T) == 2;      // bf16: scores on the tensor cores
+  constexpr int NT = (GP + 7) / 8;           // 8-head MMA tiles
+  __shared__ __align__(16) float qs[kMma ? 4 : D * GP];
   __shared__ __align__(16) float ps[kChunk][GP];
   __shared__ float red[kWarps][GP];
   __shared__ float red_acc[kWarps][4][D];      // four heads at a time
@@ -93,11 +139,26 @@ __global__ void __launch_bounds__(kThreads) dense_split_kernel(const StepParams 
   const int64_t t_end = min(t_begin + p.split_len, L);
 
   const T *qg = static_cast<const T *>(p.q) + b * p.q_sb;
-  for (int idx = tid; idx < D * GP; idx += kThreads) {
-    int i = idx / GP, g = idx % GP;
-    qs[idx] = g < G ? widen1(qg + (j0 + g) * p.q_sh + i) : 0.f;
+  uint32_t qb[kMma ? D / 16 : 1][kMma ? NT : 1][2];
+  if constexpr (kMma) {
+    // B fragments: head n = nt*8 + lane/4, columns ks*16 + (lane%4)*2 (+8)
+    const int n_lo = lane >> 2, kq = (lane & 3) * 2;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int n = nt * 8 + n_lo;
+        const uint32_t *qr = reinterpret_cast<const uint32_t *>(qg + (j0 + n) * p.q_sh);
+        qb[ks][nt][0] = n < G ? __ldg(qr + (ks * 16 + kq) / 2) : 0u;
+        qb[ks][nt][1] = n < G ? __ldg(qr + (ks * 16 + kq + 8) / 2) : 0u;
+      }
+  } else {
+    for (int idx = tid; idx < D * GP; idx += kThreads) {
+      int i = idx / GP, g = idx % GP;
+      qs[idx] = g < G ? widen1(qg + (j0 + g) * p.q_sh + i) : 0.f;
+    }
+    __syncthreads();
   }
-  __syncthreads();
 
   const T *krow0 = static_cast<const T *>(p.K) + b * p.k_sb + kh * p.k_sh;
   const T *vrow0 = static_cast<const T *>(p.V) + b * p.v_sb + (kh * VPG) * p.v_sh;
@@ -114,11 +175,23 @@ __global__ void __launch_bounds__(kThreads) dense_split_kernel(const StepParams 
     const int64_t t = base + tid;
     const bool valid = t < t_end;
     float A[GP];
-    if (valid) {
-      dense_scores<T, D, GP>(krow0 + t * D, qs, p.scale, A);
-    } else {
+    if constexpr (kMma) {
+      // scores of this warp's 32 positions into ps (rows of this warp only),
+      // then each thread takes its own position's row
+      float *sc = &ps[warp * 32][0];
+      mma_scores<D, NT>(reinterpret_cast<const uint16_t *>(krow0), base + warp * 32, t_end - 1,
+                        qb, sc, GP, lane);
+      __syncwarp();
 #pragma unroll
-      for (int g = 0; g < GP; ++g) A[g] = -INFINITY;
+      for (int g = 0; g < GP; ++g) A[g] = valid ? sc[lane * GP + g] * p.scale : -INFINITY;
+      __syncwarp();
+    } else {
+      if (valid) {
+        dense_scores<T, D, GP>(krow0 + t * D, qs, p.scale, A);
+      } else {
+#pragma unroll
+        for (int g = 0; g < GP; ++g) A[g] = -INFINITY;
+      }
     }
 #pragma unroll
     for (int g = 0; g < GP; ++g) {
