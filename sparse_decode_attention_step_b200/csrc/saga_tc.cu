@@ -56,6 +56,7 @@ struct Cfg {
   static constexpr int kStages = D == 64 ? 8 : 4;             // 128 KB of K in flight
   static constexpr int kTBufs = 2 * kRanks;                    // TMEM score buffers
   static constexpr int kTmemCols = kTBufs * kN <= 32 ? 32 : (kTBufs * kN <= 64 ? 64 : 128);
+  static_assert(kTBufs * kN <= kTmemCols, "TMEM buffers fit the allocation");
   static constexpr int kBoxes = D / 64;                        // 64-column TMA boxes per tile
   static constexpr int kBoxBytes = kTileKeys * 128;
   static constexpr int kTileBytes = kBoxes * kBoxBytes;
