@@ -4,9 +4,12 @@
 // Splits that kept nothing carry m_s = -inf and drop out; if every split is
 // empty the output row is zero.
 //
-// One CTA of 256 threads per (b, j): the split maximum is a block-wide
-// reduction, then 256 / d groups of d threads each sum every (256/d)-th split
-// for one output element, and the groups' sums are added in shared memory.
+// One CTA of 512 threads per (b, j): the split maximum is a block-wide
+// reduction, then 512 / d groups of d threads each sum every (512/d)-th split
+// for one output element (four splits' loads in flight per thread), and the
+// groups' sums are added in shared memory. With one or two sequences the
+// step plans a hundred or more splits per row, so this loop is the part of
+// the call that does not shrink with the cache.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -14,7 +17,7 @@ namespace saga {
 
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
@@ -49,11 +52,11 @@ combine_kernel(const float *__restrict__ partials, const int32_t *__restrict__ l
   const int g = tid / D, i = tid % D;
   float a = 0.f, l = 0.f;
   int cnt = 0;
+#pragma unroll 4
   for (int s = g; s < s_act; s += NG) {
     const float *r = rec + s * (D + kRecPad);
     cnt += __float_as_int(r[2]);
-    if (m == -INFINITY) continue;
-    const float w = exp2f((r[0] - m) * kLog2e);
+    const float w = m == -INFINITY ? 0.f : exp2f((r[0] - m) * kLog2e);
     l = fmaf(w, r[1], l);
     a = fmaf(w, r[kRecPad + i], a);
   }
