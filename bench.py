@@ -27,6 +27,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import subprocess
 import sys
 import time
@@ -189,9 +190,15 @@ class ClockSampler:
 
 
 def source_hash(paths):
+    """Hash of the kernel sources with comments and blank lines removed, so a
+    change of wording alone does not void counters taken on the same code."""
     h = hashlib.sha256()
     for p in paths:
-        h.update(open(p, "rb").read())
+        text = open(p, encoding="utf-8").read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        lines = [ln.rstrip() for ln in text.splitlines() if ln.strip()]
+        h.update("\n".join(lines).encode())
     return h.hexdigest()[:16]
 
 

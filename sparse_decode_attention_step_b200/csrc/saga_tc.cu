@@ -19,9 +19,17 @@
 //               and then gathers V for its own kept keys: lane group v (8
 //               lanes) owns up to four query heads that share one value
 //               head, so each kept V row is read once for all of them, and
-//               keeps their online-softmax states in registers. At the end of
-//               a unit the workers' states merge in a shared-memory tree and
-//               worker 0 writes the unit's (m, l, count, acc) records.
+//               keeps their online-softmax states in registers (rows in
+//               batches of kRows; empty rows and heads no lane group kept are
+//               skipped, and the states are rescaled only when a batch raises
+//               a maximum). At the end of a unit every worker writes its states
+//               to shared memory, the per-head weights e^{m_w - m} are formed
+//               once, and all workers write the unit's (m, l, count, acc)
+//               records.
+//
+// Modes: dump (score rows and per-row top-byte histograms of the order keys,
+// for a refresh), step (keep A >= tau), step with ties (exact top-N: keep A
+// above tau under totalOrder, and A == tau up to a per-row position).
 //
 // Query heads beyond the group (G < 16) are rows of other heads or zero rows
 // of Q; their tau is +inf, so they are never kept, and they are never dumped.
