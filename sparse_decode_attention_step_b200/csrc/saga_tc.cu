@@ -368,6 +368,7 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
     const int rank = widx >> 2;
     const int v = lane >> 3, c8 = lane & 7;
     const int hbase = pick4(hm.hbase, v), nh = pick4(hm.nh, v), vsl = pick4(hm.vs, v);
+    const bool quad = (hbase & 3) == 0 && nh == 4;   // the heads are one 16-byte quad of a row
     // two kept-score row sets, used in turn
     float *rows_base = scratch + widx * 2 * 32 * kN;
     uint32_t g = 0;
@@ -400,10 +401,18 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
           for (int cc = 0; cc < CPL; ++cc)
             raw[r][cc] = __ldg(reinterpret_cast<const uint4 *>(vrow + tr * D) + c8 + 8 * cc);
           const int ks = kk >= 0 ? kk : 0;
+          if (quad) {
+            const float4 q4 = *reinterpret_cast<const float4 *>(rows + score_slot(ks, hbase));
+            sc[r][0] = kk >= 0 ? q4.x : -INFINITY;
+            sc[r][1] = kk >= 0 ? q4.y : -INFINITY;
+            sc[r][2] = kk >= 0 ? q4.z : -INFINITY;
+            sc[r][3] = kk >= 0 ? q4.w : -INFINITY;
+          } else {
 #pragma unroll
-          for (int a = 0; a < 4; ++a) {
-            const int hd = min(hbase + a, kN - 1);
-            sc[r][a] = (kk >= 0 && a < nh) ? rows[score_slot(ks, hd)] : -INFINITY;
+            for (int a = 0; a < 4; ++a) {
+              const int hd = min(hbase + a, kN - 1);
+              sc[r][a] = (kk >= 0 && a < nh) ? rows[score_slot(ks, hd)] : -INFINITY;
+            }
           }
         }
         float mnew[4];
