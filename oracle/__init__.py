@@ -1,4 +1,5 @@
-"""Float64 CPU oracle of the SAGA + Atop-N decode attention step.
+"""Float64 CPU oracles of the SAGA + Atop-N decode attention step and of the
+closed-form GQA-to-SAGA key-head merge (``oracle.key_merge``).
 
 TEST INFRASTRUCTURE: imported only by the tests, the smoke check and the
 benchmark's CPU baseline. The product path never touches it.
