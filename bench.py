@@ -58,6 +58,9 @@ def parse():
     ap.add_argument("--dense-steps", type=int, default=8)
     ap.add_argument("--layers", type=int, default=None,
                     help="override the stack depth (same per-layer launch, smaller footprint)")
+    ap.add_argument("--merge", default=None,
+                    help="time the closed-form GQA-to-SAGA key merge on this calibration "
+                         "workload instead (synth.merge_workload.MERGE_WORKLOADS)")
     return ap.parse_args()
 
 
@@ -200,6 +203,13 @@ def source_hash(paths):
         lines = [ln.rstrip() for ln in text.splitlines() if ln.strip()]
         h.update("\n".join(lines).encode())
     return h.hexdigest()[:16]
+
+
+def step_kernel_sources():
+    """The sources the decode step's kernels and plan are built from."""
+    here = os.path.join(ROOT, "sparse_decode_attention_step_b200", "csrc")
+    return [os.path.join(here, f) for f in ("common.cuh", "sm100.cuh", "kernels.h",
+                                            "saga_api.cu", "saga_tc.cu", "combine.cu")]
 
 
 def ncu_traffic(kernel_sources):
@@ -496,9 +506,7 @@ def run_ours(args, w):
     alg_bytes = k_bytes + float(np.mean(v_bytes)) + qo_bytes
     achieved = alg_bytes / (call_ms / 1e3) / 1e9
     peak, peak_kind = measured_peaks()
-    here = os.path.join(ROOT, "sparse_decode_attention_step_b200", "csrc")
-    ksrc = [os.path.join(here, f) for f in sorted(os.listdir(here))]
-    traffic = ncu_traffic(ksrc)
+    traffic = ncu_traffic(step_kernel_sources())
 
     # ---- e2e: queries in from pinned host memory, outputs back, every step
     out_pin = torch.empty(st.out.shape, dtype=torch.float32).pin_memory()
@@ -663,8 +671,114 @@ def run_ours(args, w):
     return result
 
 
+# ---------------------------------------------------------------------------
+# the closed-form key merge (one layer's conversion)
+# ---------------------------------------------------------------------------
+MERGE_METRIC = "GQA-to-SAGA closed-form key merges/s (one layer)"
+
+
+def merge_oracle_seconds(w, X, W, Q):
+    """The float64 oracle on the host cores: one pair's Eq. (13) weight at its
+    Eq. (15) optimum, timed, scaled by the number of pairs (the matching and
+    the merged projection are negligible beside it)."""
+    from oracle import key_merge as km
+    n_pairs = w.h_k * (w.h_k - 1) // 2
+    t0 = time.perf_counter()
+    km.pair_weights(X, W, Q, w.h_q, w.h_k, w.d, 1e-6, pairs=[(0, 1)])
+    one = time.perf_counter() - t0
+    return one * n_pairs, one, n_pairs
+
+
+def bench_merge(args):
+    import torch
+    import sparse_decode_attention_step_b200 as saga
+    from synth import merge_workload as mw
+    saga.load()
+    w = mw.MERGE_WORKLOADS[args.merge]
+    Xb, Wb, Qb = mw.merge_inputs(w)
+    host = [torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).pin_memory()
+            for a in (Xb, Wb, Qb)]
+    X, W, Q = (h.cuda() for h in host)
+    ms = saga.merge_shape(w.T, w.d_model, w.h_q, w.h_k, w.d)
+    ws = saga.MergeWorkspace(ms)
+    n2 = w.h_k // 2
+    wout = torch.empty((w.h_k, w.h_k), dtype=torch.float64, device="cuda")
+    pairs = torch.empty((n2, 2), dtype=torch.int32, device="cuda")
+    total = torch.empty(1, dtype=torch.float64, device="cuda")
+    W_S = torch.empty((n2 * w.d, w.d_model), dtype=torch.float32, device="cuda")
+    outs_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (wout, pairs, W_S)]
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def call(x, wk, q):
+        saga.merge_keys(ms, x, wk, q, 1e-6, wout, pairs, W_S, ws, total=total)
+
+    for _ in range(max(3, args.warmup)):
+        call(X, W, Q)
+    torch.cuda.synchronize()
+    assert saga.read_device_error(ws) == 0
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for i in range(args.steps):
+            flush.zero_()                       # every call starts with a cold L2
+            ev[i][0].record(stream)
+            call(X, W, Q)
+            ev[i][1].record(stream)
+        # end to end: inputs in from pinned host memory, results back
+        for i in range(args.steps):
+            flush.zero_()
+            ee[i][0].record(stream)
+            X.copy_(host[0], non_blocking=True)
+            W.copy_(host[1], non_blocking=True)
+            Q.copy_(host[2], non_blocking=True)
+            call(X, W, Q)
+            for h, t in zip(outs_h, (wout, pairs, W_S)):
+                h.copy_(t, non_blocking=True)
+            ee[i][1].record(stream)
+        torch.cuda.synchronize()
+    call_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    e2e_ms = float(np.mean([a.elapsed_time(b) for a, b in ee]))
+    assert saga.read_device_error(ws) == 0
+    HD = w.h_k * w.d
+    flops = (2.0 * w.T * w.d_model * HD          # K = X W^T
+             + 3 * 2.0 * w.T * HD * HD            # C = K^T K as three bf16 products
+             + 2.0 * w.T * w.d * w.d * w.h_q)     # the S_r
+    h2d = sum(h.numel() * h.element_size() for h in host)
+    d2h = sum(h.numel() * h.element_size() for h in outs_h)
+    cpu = None
+    if not args.no_cpu_baseline:
+        Xw, Ww, Qw = (synth.widen(a) for a in (Xb, Wb, Qb))
+        secs, one, n_pairs = merge_oracle_seconds(w, Xw, Ww, Qw)
+        cpu = {"value": 1.0 / secs, "unit": "merges/s", "cores": blas_threads(),
+               "kind": "oracle",
+               "sample": f"the weight of pair (0, 1) (Eq. 13 from explicit logits at the "
+                         f"Eq. 15 optimum) timed once, {one:.2f} s, scaled by {n_pairs} pairs"}
+    line = {
+        "metric": MERGE_METRIC, "value": 1e3 / call_ms, "unit": "merges/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": call_ms,
+        "higher_is_better": True, "scaling": "none", "vs_baseline": None,
+        "dtype": "bf16 GEMMs (f32 accumulate), f64 pair algebra", "data": "synthetic",
+        "config": {"workload": w.name, "T": w.T, "d_model": w.d_model, "h_q": w.h_q,
+                   "h_k": w.h_k, "d": w.d, "l2": "flushed before every call"},
+        "gpu_launches": 8 * args.steps,
+        "gemm_tflops_algorithmic": flops / (call_ms / 1e3) / 1e12,
+        "e2e": {"value": 1e3 / e2e_ms, "unit": "merges/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "pairs": [tuple(p) for p in pairs.cpu().tolist()],
+        "clocks": clk.summary(),
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
+    if args.merge is not None:
+        bench_merge(args)
+        return
     w = synth.WORKLOADS[args.workload]
     if args.layers is not None:
         w = w.with_(layers=args.layers)

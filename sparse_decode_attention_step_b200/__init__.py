@@ -40,9 +40,15 @@ class saga_shape(ctypes.Structure):
                 ("v_stride_b", ctypes.c_int64), ("v_stride_h", ctypes.c_int64)]
 
 
+class saga_merge_shape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("d_model", ctypes.c_int32), ("h_q", ctypes.c_int32),
+                ("h_k", ctypes.c_int32), ("d", ctypes.c_int32)]
+
+
 _lib = None
 _P = ctypes.c_void_p
 _SP = ctypes.POINTER(saga_shape)
+_MP = ctypes.POINTER(saga_merge_shape)
 
 _SIGS = {
     "saga_shape_contiguous": (None, [_SP, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
@@ -63,6 +69,9 @@ _SIGS = {
     "saga_decode_step_noalloc": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P, _P, _P]),
     "saga_read_device_error": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_int32)]),
     "saga_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "saga_merge_workspace_size": (ctypes.c_size_t, [_MP]),
+    "saga_merge_keys": (ctypes.c_int, [_MP, _P, _P, _P, ctypes.c_double, _P, _P, _P, _P, _P,
+                                       ctypes.c_size_t, _P]),
 }
 
 
@@ -214,3 +223,41 @@ def read_device_error(ws, stream=None):
     if rc not in (SAGA_OK, SAGA_ERR_DEVICE):
         raise SagaError(rc, "saga_read_device_error")
     return flags.value
+
+
+# ---------------------------------------------------------------------------
+# closed-form GQA-to-SAGA key-head merge (include/saga_merge.h)
+# ---------------------------------------------------------------------------
+def merge_shape(T, d_model, h_q, h_k, d):
+    return saga_merge_shape(T, d_model, h_q, h_k, d)
+
+
+def merge_workspace_size(mshape):
+    return int(load().saga_merge_workspace_size(ctypes.byref(mshape)))
+
+
+class MergeWorkspace:
+    """Device workspace for saga_merge_keys, allocated through torch; its
+    error word is zeroed."""
+
+    def __init__(self, mshape, device="cuda", stream=None):
+        import torch
+        self.nbytes = merge_workspace_size(mshape)
+        if self.nbytes == 0:
+            raise SagaError(SAGA_ERR_INVALID_ARG, "saga_merge_workspace_size")
+        self.buf = torch.empty(self.nbytes, dtype=torch.uint8, device=device)
+        workspace_init(self.buf, self.nbytes, stream)
+
+    def data_ptr(self):
+        return self.buf.data_ptr()
+
+
+def merge_keys(mshape, X, W_K, Q, rcond, w, pairs, W_S, ws, total=None, stream=None):
+    """Pair weights w [h_k][h_k] (float64), the minimum-weight pairing
+    pairs [h_k/2][2] (int32) and the student's key projection
+    W_S [h_k/2*d][d_model] (float32) from bf16 X [T][d_model],
+    W_K [h_k*d][d_model] and Q [T][h_q*d]."""
+    p, n = _ws(ws)
+    _check(load().saga_merge_keys(ctypes.byref(mshape), _ptr(X), _ptr(W_K), _ptr(Q),
+                                  float(rcond), _ptr(w), _ptr(pairs), _ptr(total), _ptr(W_S),
+                                  p, n, _stream(stream)), "saga_merge_keys")

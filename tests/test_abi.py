@@ -131,3 +131,38 @@ def test_append_kv_host_checks(lib):
     assert call(V=ok + 8) == saga.SAGA_ERR_INVALID_ARG        # not 16-byte aligned
     assert call(ws=None) == saga.SAGA_ERR_WORKSPACE
     assert call(n=255) == saga.SAGA_ERR_WORKSPACE             # room for the error word only
+
+
+def test_merge_workspace_size(lib):
+    ok = saga.merge_shape(8192, 2048, 32, 8, 64)
+    n = saga.merge_workspace_size(ok)
+    # at least the transposed queries and the keys' hi/lo rows
+    assert n >= 8192 * 32 * 64 * 2 + 2 * 8192 * 8 * 64 * 2
+    assert n % 256 == 0
+    for bad in [dict(T=100), dict(T=64), dict(d_model=60), dict(h_k=3), dict(h_q=12),
+                dict(d=96), dict(h_k=18, h_q=36)]:
+        kw = dict(T=8192, d_model=2048, h_q=32, h_k=8, d=64)
+        kw.update(bad)
+        assert saga.merge_workspace_size(saga.merge_shape(**kw)) == 0, bad
+
+
+def test_merge_host_checks(lib):
+    s = saga.merge_shape(1024, 512, 8, 4, 64)
+    need = saga.merge_workspace_size(s)
+    ok = 1 << 40    # never dereferenced: validation fails first
+    call = lambda shp=s, **o: lib.saga_merge_keys(
+        ctypes.byref(shp), o.get("X", ok), o.get("W", ok), o.get("Q", ok), o.get("rcond", 1e-6),
+        o.get("w", ok), o.get("pairs", ok), o.get("total", None), o.get("W_S", ok),
+        o.get("ws", ok), o.get("n", need), None)
+    assert call(X=None) == saga.SAGA_ERR_INVALID_ARG
+    assert call(W=ok + 8) == saga.SAGA_ERR_INVALID_ARG        # not 16-byte aligned
+    assert call(pairs=None) == saga.SAGA_ERR_INVALID_ARG
+    assert call(rcond=-1.0) == saga.SAGA_ERR_INVALID_ARG
+    assert call(rcond=float("nan")) == saga.SAGA_ERR_INVALID_ARG
+    assert call(total=ok + 4) == saga.SAGA_ERR_INVALID_ARG    # float64 output misaligned
+    assert call(ws=None) == saga.SAGA_ERR_WORKSPACE
+    assert call(ws=ok + 128) == saga.SAGA_ERR_WORKSPACE
+    assert call(n=need - 1) == saga.SAGA_ERR_WORKSPACE
+    assert call(saga.merge_shape(1024, 512, 8, 3, 64)) == saga.SAGA_ERR_INVALID_ARG   # odd h_k
+    assert call(saga.merge_shape(1024, 512, 8, 4, 96)) == saga.SAGA_ERR_UNSUPPORTED   # d
+    assert call(saga.merge_shape(1024, 512, 36, 18, 64)) == saga.SAGA_ERR_UNSUPPORTED  # h_k > 16
