@@ -8,8 +8,9 @@
 //   3. C = K^T K over T as hi.hi + hi.lo + lo.hi, split over T (tcgen05 GEMM)
 //      S_r = sum_{j of r} Q^j^T Q^j, split over T                (tcgen05 GEMM)
 //   4. partial sums -> float64 C and S_r
-//   5. one CTA per pair (a, b): Jacobi eigen-decomposition of S_a + S_b in
-//      float64, pseudoinverse, A_a = S_a P, A_b = S_b P, w(a,b) = trace(D A_a S_b)
+//   5. one CTA per pair (a, b), float64: P = (S_a + S_b)^+ (Gauss-Jordan inverse
+//      when it provably is the pseudoinverse, else Jacobi eigen-decomposition),
+//      A_a = S_a P, A_b = S_b P, w(a,b) = trace(D A_a S_b)
 //   6. one CTA: minimum-weight perfect matching by a subset programme
 //   7. W_S rows of merged head i = (W^a A_a + W^b A_b)^T for pairs[i]
 // The GEMMs are the dense contractions (T = thousands of tokens); the
@@ -42,7 +43,7 @@ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // ---- tcgen05 GEMM ---------------------------------------------------------
 constexpr int kBM = 128, kBN = 128, kBK = 64;
-constexpr int kGStages = 4;
+constexpr int kGStages = 6;
 constexpr int kOpBytes = kBM * kBK * 2;          // one operand tile: 16 KB
 constexpr int kStageBytes = 2 * kOpBytes;
 constexpr int kGemmThreads = 192;
@@ -321,7 +322,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                                     S_sum + static_cast<size_t>(b) * D * D, C_sum,
                                     static_cast<long long>(h_k) * D, a, b, rcond, S, E, rc, rs,
                                     rowbuf, inv, Ag + static_cast<size_t>(blockIdx.x) * 2 * D * D,
-                                    nullptr);
+                                    true, nullptr);
   if (threadIdx.x == 0) {
     w[a * h_k + b] = wab;
     w[b * h_k + a] = wab;
@@ -348,40 +349,40 @@ __global__ void __launch_bounds__(kMatchThreads)
 // ---- the student's key projection ------------------------------------------------
 // W_S[i*d + c][x] = sum_m W_lin[a*d + m][x] A_a[m][c] + sum_m W_lin[b*d + m][x] A_b[m][c]
 // for (a, b) = pairs[i]; the sum runs as in merged_elem. Grid
-// (ceil(d_model / 256), d / 32, h_k / 2); a thread owns one x and 32 c.
+// (ceil(d_model / 128), d / 16, h_k / 2); a thread owns one x and 16 c.
+constexpr int kProjX = 128, kProjC = 16;
+
 template <int D>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kProjX)
     km_project_kernel(const uint16_t *__restrict__ W_lin, int d_model, int h_k,
                       const int32_t *__restrict__ pairs, const double *__restrict__ Ag,
                       float *__restrict__ W_S) {
-  __shared__ double sA[D][32];
-  const int i = blockIdx.z, c0 = blockIdx.y * 32;
+  __shared__ double sA[2][D][kProjC];
+  const int i = blockIdx.z, c0 = blockIdx.y * kProjC;
   const int a = pairs[2 * i], b = pairs[2 * i + 1];
   const double *A = Ag + static_cast<size_t>(pair_index(a, b, h_k)) * 2 * D * D;
-  const int x = blockIdx.x * 256 + threadIdx.x;
-  double acc[32];
+  for (int e = threadIdx.x; e < 2 * D * kProjC; e += blockDim.x) {
+    const int r = e / (D * kProjC), m = (e / kProjC) % D, c = e % kProjC;
+    sA[r][m][c] = A[static_cast<size_t>(r) * D * D + static_cast<size_t>(m) * D + c0 + c];
+  }
+  __syncthreads();
+  const int x = blockIdx.x * kProjX + threadIdx.x;
+  if (x >= d_model) return;
+  double acc[kProjC];
 #pragma unroll
-  for (int c = 0; c < 32; ++c) acc[c] = 0.0;
+  for (int c = 0; c < kProjC; ++c) acc[c] = 0.0;
   for (int r = 0; r < 2; ++r) {
-    __syncthreads();                      // the previous r's columns are read
-    for (int e = threadIdx.x; e < D * 32; e += blockDim.x) {
-      const int m = e / 32, c = e % 32;
-      sA[m][c] = A[static_cast<size_t>(r) * D * D + static_cast<size_t>(m) * D + c0 + c];
-    }
-    __syncthreads();
-    if (x < d_model) {
-      const uint16_t *Wr = W_lin + static_cast<size_t>(r == 0 ? a : b) * D * d_model + x;
-      for (int m = 0; m < D; ++m) {
-        const double wv = static_cast<double>(
-            __uint_as_float(static_cast<uint32_t>(Wr[static_cast<size_t>(m) * d_model]) << 16));
+    const uint16_t *Wr = W_lin + static_cast<size_t>(r == 0 ? a : b) * D * d_model + x;
+#pragma unroll 4
+    for (int m = 0; m < D; ++m) {
+      const double wv = static_cast<double>(
+          __uint_as_float(static_cast<uint32_t>(Wr[static_cast<size_t>(m) * d_model]) << 16));
 #pragma unroll
-        for (int c = 0; c < 32; ++c) acc[c] = fma(wv, sA[m][c], acc[c]);
-      }
+      for (int c = 0; c < kProjC; ++c) acc[c] = fma(wv, sA[r][m][c], acc[c]);
     }
   }
-  if (x >= d_model) return;
 #pragma unroll
-  for (int c = 0; c < 32; ++c)
+  for (int c = 0; c < kProjC; ++c)
     W_S[(static_cast<size_t>(i) * D + c0 + c) * d_model + x] = static_cast<float>(acc[c]);
 }
 
@@ -642,14 +643,14 @@ extern "C" saga_status saga_merge_keys(const saga_merge_shape *shape, const void
   if (cudaGetLastError() != cudaSuccess) return SAGA_ERR_CUDA;
   // 7. the student's key projection
   {
-    const dim3 grid(static_cast<unsigned>(ceil_div(s.d_model, 256)), static_cast<unsigned>(d / 32),
-                    static_cast<unsigned>(s.h_k / 2));
+    const dim3 grid(static_cast<unsigned>(ceil_div(s.d_model, kProjX)),
+                    static_cast<unsigned>(d / kProjC), static_cast<unsigned>(s.h_k / 2));
     if (d == 64)
-      km_project_kernel<64><<<grid, 256, 0, st>>>(static_cast<const uint16_t *>(W_K), s.d_model,
-                                                 s.h_k, pairs, Ag, W_S);
+      km_project_kernel<64><<<grid, kProjX, 0, st>>>(static_cast<const uint16_t *>(W_K),
+                                                    s.d_model, s.h_k, pairs, Ag, W_S);
     else
-      km_project_kernel<128><<<grid, 256, 0, st>>>(static_cast<const uint16_t *>(W_K), s.d_model,
-                                                  s.h_k, pairs, Ag, W_S);
+      km_project_kernel<128><<<grid, kProjX, 0, st>>>(static_cast<const uint16_t *>(W_K),
+                                                     s.d_model, s.h_k, pairs, Ag, W_S);
     if (cudaGetLastError() != cudaSuccess) return SAGA_ERR_CUDA;
   }
   return SAGA_OK;

@@ -190,6 +190,53 @@ KM_HD void pinv_from_eigen(const Team &tm, int d, const VT *E, const double *inv
   }
 }
 
+// In-place inverse of the symmetric positive definite d x d matrix S by
+// Gauss-Jordan sweeps without pivoting (the pivots of an SPD matrix are its
+// Schur complements, all positive). Step k saves column and row k (col, row
+// [d]), then updates every entry from the saved values. Returns false, with
+// S undefined, as soon as a pivot is not a positive finite number.
+KM_HD bool spd_inverse(const Team &tm, int d, double *S, double *col, double *row) {
+  for (int k = 0; k < d; ++k) {
+    for (int i = tm.tid; i < d; i += tm.n) {
+      col[i] = S[i * d + k];
+      row[i] = S[k * d + i];
+    }
+    tm.sync();
+    const double p = col[k];
+    if (!(p > 0.0) || !(p < INFINITY)) return false;   // every thread reads the same pivot
+    const double ip = 1.0 / p;
+    for (int e = tm.tid; e < d * d; e += tm.n) {
+      const int i = e / d, j = e % d;
+      double v;
+      if (i == k && j == k) v = ip;
+      else if (i == k) v = row[j] * ip;
+      else if (j == k) v = -(col[i] * ip);
+      else v = fma(-col[i], row[j] * ip, S[e]);
+      S[e] = v;
+    }
+    tm.sync();
+  }
+  return true;
+}
+
+// Whether an inverse of S (its trace `tr`) is its pseudoinverse under the
+// cutoff rcond: the smallest eigenvalue is at least 1 / ||S^-1||_F and the
+// largest at most the trace, so 1 / ||S^-1||_F > rcond * trace keeps every
+// eigenvalue. Row sums of squares in order, then the rows.
+KM_HD bool inverse_is_pinv(const Team &tm, int d, const double *Sinv, double tr, double rcond,
+                           double *rowbuf) {
+  for (int i = tm.tid; i < d; i += tm.n) {
+    double acc = 0.0;
+    for (int j = 0; j < d; ++j) acc = fma(Sinv[i * d + j], Sinv[i * d + j], acc);
+    rowbuf[i] = acc;
+  }
+  tm.sync();
+  double fro2 = 0.0;
+  for (int i = 0; i < d; ++i) fro2 += rowbuf[i];
+  tm.sync();
+  return fro2 < INFINITY && 1.0 > rcond * tr * sqrt(fro2);
+}
+
 // out = A B for d x d row-major matrices, sum over m in order.
 KM_HD void matmul_dd(const Team &tm, int d, const double *A, const double *B, double *out) {
   for (int e = tm.tid; e < d * d; e += tm.n) {
@@ -251,26 +298,43 @@ constexpr double kJacobiTol = 1e-13;   // off-diagonal norm / diagonal norm at c
 
 // Everything one pair (a, b) needs, from the query Gram matrices S_a, S_b
 // [d][d] and the key Gram matrix C [hd][hd] (all float64):
-//   S_a + S_b = E^T diag(lambda) E (Jacobi), P = (S_a + S_b)^+,
-//   A_a = S_a P and A_b = S_b P into Ag [2][d][d] (Eq. 15 is W^a A_a + W^b A_b),
-//   returns w(a, b) = trace(D A_a S_b), the Eq. (13) loss at the optimum.
+//   P = (S_a + S_b)^+, A_a = S_a P and A_b = S_b P into Ag [2][d][d]
+//   (Eq. 15 is W^a A_a + W^b A_b), and returns w(a, b) = trace(D A_a S_b), the
+//   Eq. (13) loss at the optimum.
+// P is the plain inverse when `direct` is set, the Gauss-Jordan sweeps
+// succeed and the inverse provably keeps every eigenvalue above the cutoff
+// (then it is the pseudoinverse); otherwise the Jacobi eigen-decomposition
+// gives it with the cutoff applied. *path receives 0 for the inverse, else
+// the number of Jacobi sweeps.
 // Shared scratch: S [d][d] (float64), E [d][d] (VT), rc, rs [d/2], rowbuf, inv [d].
 template <typename VT>
 KM_HD double pair_stage(const Team &tm, int d, const double *Sa, const double *Sb,
                         const double *C, long long hd, int a, int b, double rcond, double *S,
                         VT *E, double *rc, double *rs, double *rowbuf, double *inv, double *Ag,
-                        int *sweeps) {
+                        bool direct, int *path) {
   for (int e = tm.tid; e < d * d; e += tm.n) S[e] = Sa[e] + Sb[e];
   tm.sync();
-  const int sw = jacobi_eigh(tm, d, S, E, rc, rs, rowbuf, kMaxSweeps, kJacobiTol);
-  pinv_weights(tm, d, S, rcond, inv);
-  pinv_from_eigen(tm, d, E, inv, S);        // P replaces S (its diagonal was read above)
-  tm.sync();
+  bool have = false;
+  if (direct) {
+    double tr = 0.0;
+    for (int l = 0; l < d; ++l) tr += S[l * d + l];
+    tm.sync();                               // the trace is read before the sweeps
+    have = spd_inverse(tm, d, S, inv, rowbuf) && inverse_is_pinv(tm, d, S, tr, rcond, rowbuf);
+  }
+  int sw = 0;
+  if (!have) {
+    for (int e = tm.tid; e < d * d; e += tm.n) S[e] = Sa[e] + Sb[e];
+    tm.sync();
+    sw = jacobi_eigh(tm, d, S, E, rc, rs, rowbuf, kMaxSweeps, kJacobiTol);
+    pinv_weights(tm, d, S, rcond, inv);
+    pinv_from_eigen(tm, d, E, inv, S);      // P replaces S (its diagonal was read above)
+    tm.sync();
+  }
   matmul_dd(tm, d, Sa, S, Ag);
   matmul_dd(tm, d, Sb, S, Ag + d * d);
   tm.sync();
   const double w = pair_weight(tm, d, Ag, Sb, C, hd, a, b, S, rowbuf);
-  if (sweeps != nullptr && tm.tid == 0) *sweeps = sw;
+  if (path != nullptr && tm.tid == 0) *path = sw;
   return w;
 }
 

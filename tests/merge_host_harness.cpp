@@ -33,20 +33,23 @@ void km_host_rounds(int d, int32_t *out) {
     }
 }
 
-// The per-pair stage as the pair kernel runs it; vt_float selects the float
-// eigenvector storage of the d = 128 kernel. Ag receives A_a, A_b [2][d][d].
-double km_host_pair(int d, int vt_float, const double *Sa, const double *Sb, const double *C,
-                    long long hd, int a, int b, double rcond, double *Ag, int *sweeps) {
+// The per-pair stage as the pair kernel runs it (direct = 1; 0 forces the
+// eigen-decomposition); vt_float selects the float eigenvector storage of the
+// d = 128 kernel. Ag receives A_a, A_b [2][d][d]; *path 0 for the inverse,
+// else the Jacobi sweeps.
+double km_host_pair(int d, int vt_float, int direct, const double *Sa, const double *Sb,
+                    const double *C, long long hd, int a, int b, double rcond, double *Ag,
+                    int *path) {
   std::vector<double> S(d * d), rc(d / 2), rs(d / 2), rowbuf(d), inv(d);
   const Team tm{0, 1};
   if (vt_float) {
     std::vector<float> E(d * d);
     return pair_stage<float>(tm, d, Sa, Sb, C, hd, a, b, rcond, S.data(), E.data(), rc.data(),
-                             rs.data(), rowbuf.data(), inv.data(), Ag, sweeps);
+                             rs.data(), rowbuf.data(), inv.data(), Ag, direct != 0, path);
   }
   std::vector<double> E(d * d);
   return pair_stage<double>(tm, d, Sa, Sb, C, hd, a, b, rcond, S.data(), E.data(), rc.data(),
-                            rs.data(), rowbuf.data(), inv.data(), Ag, sweeps);
+                            rs.data(), rowbuf.data(), inv.data(), Ag, direct != 0, path);
 }
 
 // The matching kernel's programme on w [n][n]: pairs [n/2][2], total.

@@ -51,8 +51,9 @@ def host(tmp_path_factory):
     lib.km_host_jacobi.argtypes = [ctypes.c_int, D_P, D_P]
     lib.km_host_jacobi.restype = ctypes.c_int
     lib.km_host_rounds.argtypes = [ctypes.c_int, I_P]
-    lib.km_host_pair.argtypes = [ctypes.c_int, ctypes.c_int, D_P, D_P, D_P, ctypes.c_longlong,
-                                 ctypes.c_int, ctypes.c_int, ctypes.c_double, D_P, I_P]
+    lib.km_host_pair.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, D_P, D_P, D_P,
+                                 ctypes.c_longlong, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                 D_P, I_P]
     lib.km_host_pair.restype = ctypes.c_double
     lib.km_host_match.argtypes = [ctypes.c_int, D_P, I_P, D_P]
     lib.km_host_merged.argtypes = [ctypes.c_int, ctypes.c_int, D_P, D_P, D_P, D_P, D_P]
@@ -125,10 +126,15 @@ def gram_inputs(w):
     return X, W, Q, S, np.ascontiguousarray(C)
 
 
-@pytest.mark.parametrize("name,vt_float,rtol", [
-    ("merge_tiny", 0, 1e-9), ("merge_tail_g1", 0, 1e-9), ("merge_tiny_d128", 0, 1e-9),
-    ("merge_tiny_d128", 1, 1e-5), ("merge_rank_deficient", 0, 1e-9)])
-def test_pair_stage_against_oracle(host, name, vt_float, rtol):
+@pytest.mark.parametrize("name,vt_float,direct,rtol", [
+    ("merge_tiny", 0, 1, 1e-9), ("merge_tiny", 0, 0, 1e-9), ("merge_tail_g1", 0, 1, 1e-9),
+    ("merge_tiny_d128", 0, 0, 1e-9), ("merge_tiny_d128", 1, 0, 1e-5),
+    ("merge_tiny_d128", 1, 1, 1e-9), ("merge_rank_deficient", 0, 1, 1e-9)])
+def test_pair_stage_against_oracle(host, name, vt_float, direct, rtol):
+    """Both ways to the pseudoinverse: the Gauss-Jordan inverse where it
+    provably equals it (full-rank calibration sets), the Jacobi
+    eigen-decomposition otherwise (forced with direct = 0, and taken by
+    itself on the rank-deficient set)."""
     w = mw.MERGE_WORKLOADS[name]
     X, W, Q, S, C = gram_inputs(w)
     d, n = w.d, w.h_k
@@ -137,10 +143,14 @@ def test_pair_stage_against_oracle(host, name, vt_float, rtol):
         for b in range(a + 1, n):
             Ag = np.zeros((2, d, d))
             sw = np.zeros(1, np.int32)
-            got = host.km_host_pair(d, vt_float, dptr(np.ascontiguousarray(S[a])),
+            got = host.km_host_pair(d, vt_float, direct, dptr(np.ascontiguousarray(S[a])),
                                     dptr(np.ascontiguousarray(S[b])), dptr(C), n * d, a, b,
                                     1e-6, dptr(Ag), iptr(sw))
             assert got == pytest.approx(ref_w[a, b], rel=rtol)
+            if direct and w.d_eff is None:
+                assert sw[0] == 0                      # full rank: the inverse was taken
+            else:
+                assert sw[0] >= 1                      # the eigen-decomposition ran
             out = np.zeros((d, w.d_model))
             Wa = np.ascontiguousarray(W[a * d:(a + 1) * d])
             Wb = np.ascontiguousarray(W[b * d:(b + 1) * d])
