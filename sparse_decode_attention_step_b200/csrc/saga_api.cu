@@ -16,6 +16,7 @@ constexpr int64_t kSms = 148;              // B200 SMs: the persistent grid
 constexpr int64_t kTileKeys = 128;         // split lengths are multiples of a K tile
 constexpr int64_t kUnitTiles = 32;         // grid-per-split kernels: at most about this many tiles per split
 constexpr int64_t kPersistTiles = 128;     // persistent kernel: at most about this many tiles per unit
+constexpr int64_t kGridCtasPerSm = 4;      // grid-per-split kernels: at least this many units per SM
 constexpr size_t kAlign = 256;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -31,7 +32,9 @@ bool use_tc(const saga_shape &s);
 
 // Splits of equal length, a multiple of the K tile.
 // Grid-per-split kernels (SIMT, dense): the (b, kh, split) units number about a
-// whole multiple of the SM count, with at most about kUnitTiles tiles each.
+// whole multiple of the SM count, with at most about kUnitTiles tiles each and
+// at least kGridCtasPerSm per SM where the sequence is long enough, since
+// those kernels hide their load latency only with several CTAs per SM.
 // Persistent tensor-core kernel: at most one unit per SM and wave, units of up
 // to about kPersistTiles tiles, since every unit ends with a merge of the
 // workers' states.
@@ -46,7 +49,7 @@ Plan make_plan(const saga_shape &s, bool persistent) {
     s_target = std::max<int64_t>(1, kSms * waves / rows);
   } else {
     const int64_t waves = std::max<int64_t>(1, ceil_div(tiles, kSms * kUnitTiles));
-    s_target = std::max<int64_t>(1, ceil_div(kSms * waves, rows));
+    s_target = std::max<int64_t>(1, ceil_div(kSms * std::max(waves, kGridCtasPerSm), rows));
   }
   p.split_len = ceil_div(ceil_div(L, s_target), kTileKeys) * kTileKeys;
   p.S = static_cast<int>(ceil_div(L, p.split_len));
