@@ -297,11 +297,47 @@ static cudaError_t launch_dd(const StepParams &p, int gp, int vpg, dim3 grid, cu
   }
 }
 
+template <typename T, int D, int VPG>
+static const void *kernel_dv(int gp) {
+  switch (gp) {
+    case 4: return reinterpret_cast<const void *>(dense_split_kernel<T, D, 4, VPG>);
+    case 8: return reinterpret_cast<const void *>(dense_split_kernel<T, D, 8, VPG>);
+    case 12: return reinterpret_cast<const void *>(dense_split_kernel<T, D, 12, VPG>);
+    case 16: return reinterpret_cast<const void *>(dense_split_kernel<T, D, 16, VPG>);
+    default: return nullptr;
+  }
+}
+
+template <typename T, int D>
+static const void *kernel_dd(int gp, int vpg) {
+  switch (vpg) {
+    case 1: return kernel_dv<T, D, 1>(gp);
+    case 2: return kernel_dv<T, D, 2>(gp);
+    case 4: return kernel_dv<T, D, 4>(gp);
+    default: return nullptr;
+  }
+}
+
 bool dense_supports(int h_q, int h_k, int h_v) {
   if (h_k < 1 || h_v % h_k != 0 || h_q % h_v != 0) return false;
   const int G = h_q / h_k, vpg = h_v / h_k;
   if (vpg == 1) return G <= 16;
   return (vpg == 2 || vpg == 4) && (G == 4 || G == 8 || G == 12 || G == 16) && G % vpg == 0;
+}
+
+int dense_ctas_per_sm(int dtype, int d, int h_q, int h_k, int h_v) {
+  if (!dense_supports(h_q, h_k, h_v)) return 0;
+  const int G = h_q / h_k, vpg = h_v / h_k;
+  const int gp = vpg == 1 ? (G + 3) / 4 * 4 : G;
+  const void *k = nullptr;
+  if (dtype == SAGA_BF16)
+    k = d == 64 ? kernel_dd<uint16_t, 64>(gp, vpg) : d == 128 ? kernel_dd<uint16_t, 128>(gp, vpg) : nullptr;
+  else
+    k = d == 64 ? kernel_dd<float, 64>(gp, vpg) : d == 128 ? kernel_dd<float, 128>(gp, vpg) : nullptr;
+  int n = 0;
+  if (k == nullptr || cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, kThreads, 0) != cudaSuccess)
+    return 0;
+  return n;
 }
 
 cudaError_t launch_dense_split(const StepParams &p, int dtype, int d, cudaStream_t st) {

@@ -44,6 +44,8 @@ cudaError_t launch_radix_select(const float *scores, int64_t row_stride, const i
 // h_q / h_k <= 16) or SAGA heads (h_v / h_k in {2, 4}, h_q / h_k in {4, 8, 12, 16}).
 bool dense_supports(int h_q, int h_k, int h_v);
 cudaError_t launch_dense_split(const StepParams &p, int dtype, int d, cudaStream_t st);
+// CTAs of the shape's dense kernel that fit one SM (0 if unknown).
+int dense_ctas_per_sm(int dtype, int d, int h_q, int h_k, int h_v);
 
 // KV-cache append over grid (B): rows k_new [B][h_k][d] and v_new [B][h_v][d]
 // (contiguous) to position l_kv[b], then l_kv[b] += 1. Strides in elements.

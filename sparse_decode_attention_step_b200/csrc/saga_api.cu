@@ -32,13 +32,15 @@ bool use_tc(const saga_shape &s);
 
 // Splits of equal length, a multiple of the K tile.
 // Grid-per-split kernels (SIMT, dense): the (b, kh, split) units number about a
-// whole multiple of the SM count, with at most about kUnitTiles tiles each and
-// at least kGridCtasPerSm per SM where the sequence is long enough, since
-// those kernels hide their load latency only with several CTAs per SM.
+// whole multiple of the SM count, with at most about kUnitTiles tiles each and,
+// where the sequence is long enough, at least as many per SM as fit on one
+// (`ctas_per_sm`, at most kGridCtasPerSm, which sizes the workspace): those
+// kernels hide their load latency only with every resident slot filled, and
+// more splits than slots only add waves and combine work.
 // Persistent tensor-core kernel: at most one unit per SM and wave, units of up
 // to about kPersistTiles tiles, since every unit ends with a merge of the
 // workers' states.
-Plan make_plan(const saga_shape &s, bool persistent) {
+Plan make_plan(const saga_shape &s, bool persistent, int64_t ctas_per_sm = kGridCtasPerSm) {
   Plan p{};
   const int64_t rows = static_cast<int64_t>(s.B) * s.h_k;
   const int64_t L = std::max<int64_t>(1, s.max_l_kv);
@@ -49,7 +51,8 @@ Plan make_plan(const saga_shape &s, bool persistent) {
     s_target = std::max<int64_t>(1, kSms * waves / rows);
   } else {
     const int64_t waves = std::max<int64_t>(1, ceil_div(tiles, kSms * kUnitTiles));
-    s_target = std::max<int64_t>(1, ceil_div(kSms * std::max(waves, kGridCtasPerSm), rows));
+    const int64_t slots = std::min(std::max<int64_t>(1, ctas_per_sm), kGridCtasPerSm);
+    s_target = std::max<int64_t>(1, ceil_div(kSms * std::max(waves, slots), rows));
   }
   p.split_len = ceil_div(ceil_div(L, s_target), kTileKeys) * kTileKeys;
   p.S = static_cast<int>(ceil_div(L, p.split_len));
@@ -162,7 +165,7 @@ saga_status run_dense(const saga_shape &s, const void *q, const void *K, const v
   if (V == nullptr || !aligned(V, 16) || out == nullptr || !aligned(out, 16))
     return SAGA_ERR_INVALID_ARG;
   if ((r = check_ws(s, ws, ws_bytes)) != SAGA_OK) return r;
-  const Plan pl = make_plan(s, false);
+  const Plan pl = make_plan(s, false, dense_ctas_per_sm(s.dtype, s.d, s.h_q, s.h_k, s.h_v));
   StepParams p = base_params(s, pl, q, K, V, l_kv, ws);
   cudaError_t e = launch_dense_split(p, s.dtype, s.d, st);
   if (e != cudaSuccess) return SAGA_ERR_CUDA;
