@@ -212,3 +212,30 @@ def test_pair_index_round_trip(host):
                 host.km_host_pair_of(idx, n, iptr(ab))
                 assert tuple(ab) == (a, b)
                 idx += 1
+
+
+@pytest.mark.parametrize("lam_min_rel,expect_direct", [(1e-2, True), (3e-7, False), (0.0, False)])
+def test_pseudoinverse_route_and_cutoff(host, lam_min_rel, expect_direct):
+    """The plain inverse is taken only when no eigenvalue can reach the
+    cutoff rcond * lambda_max; otherwise the eigen-decomposition applies the
+    cutoff. Either way A_a = S_a (S_a + S_b)^+ matches numpy's pinv with the
+    same rcond (S_b = 0 here, so A_a is the projector onto the kept
+    eigenvectors)."""
+    rng = np.random.default_rng(41)
+    d, rcond = 64, 1e-6
+    Qm, _ = np.linalg.qr(rng.standard_normal((d, d)))
+    lam = np.exp(rng.uniform(0.0, 2.0, d))
+    lam[0] = lam_min_rel * lam.max()
+    Sa = np.ascontiguousarray((Qm * lam) @ Qm.T)
+    Sa = 0.5 * (Sa + Sa.T)
+    Sb = np.zeros((d, d))
+    C = np.zeros((2 * d, 2 * d))
+    Ag = np.zeros((2, d, d))
+    sw = np.zeros(1, np.int32)
+    got = host.km_host_pair(d, 0, 1, dptr(Sa), dptr(Sb), dptr(C), 2 * d, 0, 1, rcond, dptr(Ag),
+                            iptr(sw))
+    assert got == 0.0                                   # D = 0: nothing to lose
+    assert (sw[0] == 0) == expect_direct
+    ref = Sa @ np.linalg.pinv(Sa, rcond=rcond, hermitian=True)
+    np.testing.assert_allclose(Ag[0], ref, rtol=0, atol=1e-9)
+    np.testing.assert_array_equal(Ag[1], 0.0)
