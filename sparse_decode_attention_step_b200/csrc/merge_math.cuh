@@ -178,15 +178,49 @@ KM_HD void pinv_weights(const Team &tm, int d, const double *S, double rcond, do
   tm.sync();
 }
 
+// The d x d products below are formed in 4 x 4 blocks per item (d a
+// multiple of 4): each loaded operand value feeds four FMAs. Every element is
+// still one sum over m (or l) in increasing order.
+constexpr int kBlk = 4;
+
 // P = E^T diag(inv) E, i.e. P[i][k] = sum_l inv_l E[l][i] E[l][k].
 template <typename VT>
 KM_HD void pinv_from_eigen(const Team &tm, int d, const VT *E, const double *inv, double *P) {
-  for (int e = tm.tid; e < d * d; e += tm.n) {
-    const int i = e / d, k = e % d;
-    double acc = 0.0;
-    for (int l = 0; l < d; ++l)
-      acc = fma(inv[l] * static_cast<double>(E[l * d + i]), static_cast<double>(E[l * d + k]), acc);
-    P[e] = acc;
+  const int nb = d / kBlk;
+  for (int e = tm.tid; e < nb * nb; e += tm.n) {
+    const int i0 = (e / nb) * kBlk, k0 = (e % nb) * kBlk;
+    double acc[kBlk][kBlk];
+    for (int r = 0; r < kBlk; ++r)
+      for (int c = 0; c < kBlk; ++c) acc[r][c] = 0.0;
+    for (int l = 0; l < d; ++l) {
+      double x[kBlk], y[kBlk];
+      for (int r = 0; r < kBlk; ++r) x[r] = inv[l] * static_cast<double>(E[l * d + i0 + r]);
+      for (int c = 0; c < kBlk; ++c) y[c] = static_cast<double>(E[l * d + k0 + c]);
+      for (int r = 0; r < kBlk; ++r)
+        for (int c = 0; c < kBlk; ++c) acc[r][c] = fma(x[r], y[c], acc[r][c]);
+    }
+    for (int r = 0; r < kBlk; ++r)
+      for (int c = 0; c < kBlk; ++c) P[(i0 + r) * d + k0 + c] = acc[r][c];
+  }
+}
+
+// out = A B for d x d row-major matrices, sum over m in order.
+KM_HD void matmul_dd(const Team &tm, int d, const double *A, const double *B, double *out) {
+  const int nb = d / kBlk;
+  for (int e = tm.tid; e < nb * nb; e += tm.n) {
+    const int i0 = (e / nb) * kBlk, k0 = (e % nb) * kBlk;
+    double acc[kBlk][kBlk];
+    for (int r = 0; r < kBlk; ++r)
+      for (int c = 0; c < kBlk; ++c) acc[r][c] = 0.0;
+    for (int m = 0; m < d; ++m) {
+      double x[kBlk], y[kBlk];
+      for (int r = 0; r < kBlk; ++r) x[r] = A[(i0 + r) * d + m];
+      for (int c = 0; c < kBlk; ++c) y[c] = B[m * d + k0 + c];
+      for (int r = 0; r < kBlk; ++r)
+        for (int c = 0; c < kBlk; ++c) acc[r][c] = fma(x[r], y[c], acc[r][c]);
+    }
+    for (int r = 0; r < kBlk; ++r)
+      for (int c = 0; c < kBlk; ++c) out[(i0 + r) * d + k0 + c] = acc[r][c];
   }
 }
 
@@ -237,16 +271,6 @@ KM_HD bool inverse_is_pinv(const Team &tm, int d, const double *Sinv, double tr,
   return fro2 < INFINITY && 1.0 > rcond * tr * sqrt(fro2);
 }
 
-// out = A B for d x d row-major matrices, sum over m in order.
-KM_HD void matmul_dd(const Team &tm, int d, const double *A, const double *B, double *out) {
-  for (int e = tm.tid; e < d * d; e += tm.n) {
-    const int i = e / d, k = e % d;
-    double acc = 0.0;
-    for (int m = 0; m < d; ++m) acc = fma(A[i * d + m], B[m * d + k], acc);
-    out[e] = acc;
-  }
-}
-
 // D[k][i] of the pair (a, b) from the key Gram matrix C [hd][hd]
 // (C = K^T K, K = [K_0 ... K_{h_k-1}]): (K_a - K_b)^T (K_a - K_b).
 KM_HD double pair_gap(const double *C, long long hd, int d, int a, int b, int k, int i) {
@@ -256,16 +280,27 @@ KM_HD double pair_gap(const double *C, long long hd, int d, int a, int b, int k,
 }
 
 // Pair weight trace(D H) with H = A_a S_b (A_a = S_a (S_a + S_b)^+):
-// item (k, i) forms H[k][i] and D[i][k] H[k][i] (D symmetric, read as D[k][i])
-// into T; rows of T are summed in order, then the rows.
+// items form 4 x 4 blocks of H[k][i] and D[i][k] H[k][i] (D symmetric, read as
+// D[k][i]) into T; rows of T are summed in order, then the rows.
 KM_HD double pair_weight(const Team &tm, int d, const double *A_a, const double *S_b,
                          const double *C, long long hd, int a, int b, double *T,
                          double *rowbuf) {
-  for (int e = tm.tid; e < d * d; e += tm.n) {
-    const int k = e / d, i = e % d;
-    double h = 0.0;
-    for (int m = 0; m < d; ++m) h = fma(A_a[k * d + m], S_b[m * d + i], h);
-    T[e] = pair_gap(C, hd, d, a, b, k, i) * h;
+  const int nb = d / kBlk;
+  for (int e = tm.tid; e < nb * nb; e += tm.n) {
+    const int k0 = (e / nb) * kBlk, i0 = (e % nb) * kBlk;
+    double h[kBlk][kBlk];
+    for (int r = 0; r < kBlk; ++r)
+      for (int c = 0; c < kBlk; ++c) h[r][c] = 0.0;
+    for (int m = 0; m < d; ++m) {
+      double x[kBlk], y[kBlk];
+      for (int r = 0; r < kBlk; ++r) x[r] = A_a[(k0 + r) * d + m];
+      for (int c = 0; c < kBlk; ++c) y[c] = S_b[m * d + i0 + c];
+      for (int r = 0; r < kBlk; ++r)
+        for (int c = 0; c < kBlk; ++c) h[r][c] = fma(x[r], y[c], h[r][c]);
+    }
+    for (int r = 0; r < kBlk; ++r)
+      for (int c = 0; c < kBlk; ++c)
+        T[(k0 + r) * d + i0 + c] = pair_gap(C, hd, d, a, b, k0 + r, i0 + c) * h[r][c];
   }
   tm.sync();
   for (int k = tm.tid; k < d; k += tm.n) {
