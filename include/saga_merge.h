@@ -53,9 +53,11 @@ extern "C" {
  *                               key head r's keys are X W_K[r*d:(r+1)*d]^T
  *   Q      [T][h_q * d]         calibration queries; Q^j = columns j*d..j*d+d
  *   Query head j belongs to teacher key head floor(j * h_k / h_q).
- * Requirements: T >= 1 and T % 8 == 0; d_model >= 8 and d_model % 8 == 0;
- * h_k even, 2 <= h_k <= 16; h_q % h_k == 0; d in {64, 128}. X, W_K and Q
- * 16-byte aligned.
+ * Requirements (SAGA_ERR_INVALID_ARG otherwise): T >= 128 and T % 8 == 0;
+ * d_model >= 64 and d_model % 8 == 0 (row strides and tile boxes of the
+ * tensor-memory copies); h_k even, h_k >= 2; h_q % h_k == 0. Supported
+ * (SAGA_ERR_UNSUPPORTED otherwise): d in {64, 128}; h_k <= 16;
+ * T <= 2^21; d_model <= 2^20; h_q * d <= 2^20. X, W_K and Q 16-byte aligned.
  */
 typedef struct saga_merge_shape {
   int32_t T, d_model, h_q, h_k, d;

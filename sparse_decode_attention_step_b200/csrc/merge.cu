@@ -479,9 +479,11 @@ bool valid_shape(const saga_merge_shape *s) {
          s->h_q % s->h_k == 0 && s->d > 0;
 }
 
+// Sizes the kernels' index types and grids take: the transpose grid spans
+// T / 64 rows of blocks (at most 65535), the subset table 2^h_k entries.
 bool supported_shape(const saga_merge_shape *s) {
   return (s->d == 64 || s->d == 128) && s->h_k <= 16 &&
-         static_cast<int64_t>(s->h_q) * s->d <= (1 << 20) && s->T <= (1 << 24) &&
+         static_cast<int64_t>(s->h_q) * s->d <= (1 << 20) && s->T <= (1 << 21) &&
          s->d_model <= (1 << 20);
 }
 

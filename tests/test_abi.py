@@ -166,3 +166,5 @@ def test_merge_host_checks(lib):
     assert call(saga.merge_shape(1024, 512, 8, 3, 64)) == saga.SAGA_ERR_INVALID_ARG   # odd h_k
     assert call(saga.merge_shape(1024, 512, 8, 4, 96)) == saga.SAGA_ERR_UNSUPPORTED   # d
     assert call(saga.merge_shape(1024, 512, 36, 18, 64)) == saga.SAGA_ERR_UNSUPPORTED  # h_k > 16
+    assert call(saga.merge_shape((1 << 21) + 8, 512, 8, 4, 64)) == saga.SAGA_ERR_UNSUPPORTED
+    assert call(saga.merge_shape(120, 512, 8, 4, 64)) == saga.SAGA_ERR_INVALID_ARG     # T < 128
