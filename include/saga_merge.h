@@ -55,7 +55,7 @@ extern "C" {
  *   Query head j belongs to teacher key head floor(j * h_k / h_q).
  * Requirements (SAGA_ERR_INVALID_ARG otherwise): T >= 128 and T % 8 == 0;
  * d_model >= 64 and d_model % 8 == 0 (row strides and tile boxes of the
- * tensor-memory copies); h_k even, h_k >= 2; h_q % h_k == 0. Supported
+ * TMA copies); h_k even, h_k >= 2; h_q % h_k == 0. Supported
  * (SAGA_ERR_UNSUPPORTED otherwise): d in {64, 128}; h_k <= 16;
  * T <= 2^21; d_model <= 2^20; h_q * d <= 2^20. X, W_K and Q 16-byte aligned.
  */
@@ -85,7 +85,7 @@ size_t saga_merge_workspace_size(const saga_merge_shape *shape);
  *   total      nullable [1] float64: the matching's summed weight.
  *   W_S        [h_k / 2 * d][d_model] float32, written.
  * Errors: SAGA_ERR_INVALID_ARG for null or misaligned pointers, a bad shape
- * or rcond; SAGA_ERR_UNSUPPORTED for d outside {64, 128} or h_k > 16;
+ * or rcond; SAGA_ERR_UNSUPPORTED for a shape outside the supported sizes;
  * SAGA_ERR_WORKSPACE for a missing, misaligned or short workspace;
  * SAGA_ERR_CUDA if a launch fails.
  */
