@@ -1,0 +1,79 @@
+"""Host logic of bench.py that needs no GPU: the traffic counters are used
+only on the sources they were taken on, the hash ignores comments, the peak
+comes from the measured file, launch counts and the JSON config."""
+import importlib.util
+import json
+import os
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def bench():
+    spec = importlib.util.spec_from_file_location("bench", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_source_hash_ignores_comments_only(bench, tmp_path):
+    a = tmp_path / "a.cu"
+    a.write_text("int f() {\n  return 1;  // one\n}\n/* block\n comment */\n")
+    b = tmp_path / "b.cu"
+    b.write_text("// header\nint f() {\n\n  return 1;   \n}\n")
+    c = tmp_path / "c.cu"
+    c.write_text("int f() {\n  return 2;\n}\n")
+    assert bench.source_hash([str(a)]) == bench.source_hash([str(b)])
+    assert bench.source_hash([str(a)]) != bench.source_hash([str(c)])
+
+
+def test_step_kernel_sources_exist(bench):
+    for p in bench.step_kernel_sources():
+        assert os.path.exists(p), p
+
+
+def test_committed_traffic(bench):
+    """When the committed counters were taken on the current step-kernel
+    sources, the bench reports them, and they are about the algorithmic bytes
+    of a call (no re-reads). After a kernel change they are dropped until
+    taken again."""
+    t = bench.ncu_traffic(bench.step_kernel_sources())
+    if t is None:
+        pytest.skip("counters were taken on other kernel sources")
+    d = json.load(open(os.path.join(ROOT, "profiles", "ncu_traffic.json")))
+    assert t == d["dram_bytes_per_call"]
+    assert 0.9 < t / 341.8e6 < 1.1
+
+
+def test_traffic_is_dropped_when_sources_change(bench, tmp_path):
+    src = tmp_path / "k.cu"
+    src.write_text("int k;\n")
+    assert bench.ncu_traffic([str(src)]) is None
+
+
+def test_measured_peak(bench):
+    gbs, kind = bench.measured_peaks()
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        assert kind == "measured" and gbs == float(json.load(open(p))["hbm_gbs"])
+    else:
+        assert kind == "fallback" and gbs == bench.FALLBACK_HBM_GBS
+
+
+def test_launch_counts(bench):
+    assert bench.kernels_per_call(dense=True, refresh=False) == 2
+    assert bench.kernels_per_call(dense=False, refresh=False) == 2
+    assert bench.kernels_per_call(dense=False, refresh=True) == 4
+
+
+def test_aggregate_and_config(bench):
+    import synth
+    w = synth.WORKLOADS["llama1b_stack16_b8_128k"]
+    assert bench.aggregate_value(64, 1000.0, 1) == pytest.approx(64.0)
+    assert bench.aggregate_value(64, 1000.0, 4) == pytest.approx(256.0)
+    cfg = bench.workload_config(w, 2)
+    assert cfg["workload"] == w.name and cfg["global_batch"] == 2 * w.B
+    assert bench.rank_workload(w, 0) is w
+    assert bench.rank_workload(w, 1).seed != w.seed
