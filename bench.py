@@ -30,6 +30,7 @@ import os
 import re
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -146,7 +147,9 @@ class ClockSampler:
     def __init__(self, index):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{index}.csv")
+        # raw samples; the JSON line carries their summary
+        self.path = os.environ.get("SAGA_CLOCK_LOG") or os.path.join(
+            tempfile.gettempdir(), f"saga_clocks_gpu{index}.csv")
 
     def __enter__(self):
         try:
