@@ -270,6 +270,13 @@ saga_status saga_read_device_error(void *ws, saga_stream_t stream,
 /* Static description of a status code. */
 const char *saga_status_string(saga_status status);
 
+/* The last CUDA failure seen by a call of this library on the calling
+ * thread, as "<launch or call>: <CUDA error name> (<description>)", or the
+ * empty string if there was none. Every call that returns SAGA_ERR_CUDA
+ * records it first; a later success does not clear it. The string belongs
+ * to the library and stays valid until the thread's next failing call. */
+const char *saga_last_error(void);
+
 #ifdef __cplusplus
 }
 #endif

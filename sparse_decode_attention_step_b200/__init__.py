@@ -28,7 +28,10 @@ DEVERR_LKV_TOO_LONG = 2
 class SagaError(RuntimeError):
     def __init__(self, status, where):
         self.status = status
-        super().__init__(f"{where}: {status_string(status)} (status {status})")
+        msg = f"{where}: {status_string(status)} (status {status})"
+        if status == SAGA_ERR_CUDA:
+            msg += f": {last_error()}"
+        super().__init__(msg)
 
 
 class saga_shape(ctypes.Structure):
@@ -69,6 +72,7 @@ _SIGS = {
     "saga_decode_step_noalloc": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P, _P, _P]),
     "saga_read_device_error": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_int32)]),
     "saga_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "saga_last_error": (ctypes.c_char_p, []),
     "saga_merge_workspace_size": (ctypes.c_size_t, [_MP]),
     "saga_merge_keys": (ctypes.c_int, [_MP, _P, _P, _P, ctypes.c_double, _P, _P, _P, _P, _P,
                                        ctypes.c_size_t, _P]),
@@ -116,6 +120,11 @@ def _check(rc, where):
 
 def status_string(status):
     return load().saga_status_string(status).decode()
+
+
+def last_error():
+    """The last CUDA failure a library call saw on this thread (or "")."""
+    return load().saga_last_error().decode()
 
 
 def shape(B, h_q, h_k, h_v, d, dtype, cap, max_l_kv=None):

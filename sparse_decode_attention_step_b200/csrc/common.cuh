@@ -89,3 +89,17 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 }  // namespace saga
+
+namespace saga {
+
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start while the previous kernel in the stream is still
+// running; pdl_wait blocks until that kernel has completed and its memory
+// is visible, so nothing the previous kernel writes is read before it.
+// pdl_trigger lets the next kernel in the stream begin its own launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+}  // namespace saga

@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "common.cuh"
 
 namespace saga {
@@ -17,12 +19,18 @@ cudaError_t launch_saga_split(const StepParams &p, int mode, int dtype, int d, i
                               cudaStream_t st);
 
 // Persistent tensor-core split kernel: dump and step modes, bit-identical
-// scores between the two. Shapes it takes: saga_tc_supports.
+// scores between the two; the step modes read stored score rows instead of K
+// when p.scores_in is set. Shapes it takes: saga_tc_supports.
 cudaError_t launch_saga_tc(const StepParams &p, int mode, int d, cudaStream_t st);
 
 // bf16 caches, d in {64, 128}, G = h_q / h_k <= 16, and the query heads of a
 // group fit four lane groups: (h_v / h_k) * ceil((h_q / h_v) / 4) <= 4.
 bool saga_tc_supports(int dtype, int d, int h_q, int h_k, int h_v);
+
+// The tensor-core step kernel can stream stored score rows (StepParams::
+// scores_in, [B][h_q][row_stride] fp32) in place of K: 16-byte aligned rows
+// whose stride is a multiple of four floats.
+bool saga_tc_scores_streamable(const float *rows, int64_t row_stride);
 
 // Merge the per-split states of every (b, j) into out and sel_count.
 cudaError_t launch_combine(const float *partials, const int32_t *l_kv, int32_t *err,
@@ -54,11 +62,45 @@ cudaError_t launch_append(const void *k_new, const void *v_new, void *K, void *V
                           int64_t k_sh, int64_t v_sb, int64_t v_sh, int64_t cap,
                           cudaStream_t st);
 
+// Record a failed CUDA call for saga_last_error (per calling thread) and
+// return SAGA_ERR_CUDA; `where` names the launch or call that failed.
+saga_status cuda_fail(cudaError_t e, const char *where);
+// SAGA_OK for cudaSuccess, else cuda_fail(e, where).
+inline saga_status cuda_check(cudaError_t e, const char *where) {
+  return e == cudaSuccess ? SAGA_OK : cuda_fail(e, where);
+}
+
 // Plain step with a caller-chosen scratch buffer (see saga_decode_step_noalloc).
 size_t plain_step_scratch_bytes(const saga_shape &s);
 saga_status plain_step_with_scratch(const saga_shape *shape, const void *q, const void *K,
                                     const void *V, const int32_t *l_kv, const float *tau,
                                     float *out, int32_t *sel_count, void *scratch,
                                     size_t scratch_bytes, cudaStream_t st);
+
+}  // namespace saga
+
+namespace saga {
+
+// Launch `kernel` on `st` with programmatic stream serialisation, so its
+// blocks may start (and run up to pdl_wait) while the previous kernel in the
+// stream finishes. Every kernel launched this way calls pdl_wait before it
+// reads or writes memory that an earlier launch in the stream may touch.
+// On the legacy default stream, which synchronises with every other stream,
+// the launch is an ordinary one (pdl_wait then returns at once).
+template <typename... P, typename... A>
+cudaError_t launch_pdl(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, A &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = (st == nullptr || st == cudaStreamLegacy) ? 0 : 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
+}
 
 }  // namespace saga

@@ -28,6 +28,7 @@
 #include <algorithm>
 #include <atomic>
 
+#include "kernels.h"
 #include "merge_math.cuh"
 #include "saga.h"
 #include "saga_merge.h"
@@ -518,6 +519,7 @@ bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 }  // namespace saga
 
 using namespace saga::merge;
+using saga::cuda_fail;
 
 extern "C" size_t saga_merge_workspace_size(const saga_merge_shape *shape) {
   if (!valid_shape(shape) || !supported_shape(shape)) return 0;
@@ -540,7 +542,7 @@ extern "C" saga_status saga_merge_keys(const saga_merge_shape *shape, const void
   const MergePlan p = make_plan(s);
   if (ws == nullptr || !aligned(ws, kAlign) || ws_bytes < p.total) return SAGA_ERR_WORKSPACE;
   EncodeTiledFn enc = encode_fn();
-  if (enc == nullptr) return SAGA_ERR_CUDA;
+  if (enc == nullptr) return cuda_fail(cudaErrorNotSupported, "cuTensorMapEncodeTiled entry point");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   char *wsb = static_cast<char *>(ws);
   int32_t *err = reinterpret_cast<int32_t *>(wsb);
@@ -559,14 +561,14 @@ extern "C" saga_status saga_merge_keys(const saga_merge_shape *shape, const void
   if (!make_map(enc, &xmap, X, s.d_model, T) || !make_map(enc, &wmap, W_K, s.d_model, HD) ||
       !make_map(enc, &ktmap, Kt, T, 2 * static_cast<int64_t>(HD)) ||
       !make_map(enc, &qtmap, Qt, T, static_cast<int64_t>(s.h_q) * d))
-    return SAGA_ERR_CUDA;
+    return cuda_fail(cudaErrorInvalidValue, "cuTensorMapEncodeTiled (key merge)");
 
   // 1. Qt = Q^T
   {
     const dim3 grid(static_cast<unsigned>(ceil_div(static_cast<int64_t>(s.h_q) * d, 64)),
                     static_cast<unsigned>(ceil_div(T, 64)));
     km_transpose_kernel<<<grid, 256, 0, st>>>(static_cast<const uint16_t *>(Q), T, s.h_q * d, Qt);
-    if (cudaGetLastError() != cudaSuccess) return SAGA_ERR_CUDA;
+    if (const cudaError_t e = cudaGetLastError(); e != cudaSuccess) return cuda_fail(e, "transpose kernel");
   }
   // 2. Kt[n][t] = (X W^T)[t][n] as bf16 hi and lo rows
   {
@@ -583,7 +585,7 @@ extern "C" saga_status saga_merge_keys(const saga_merge_shape *shape, const void
     g.lo_off = static_cast<long long>(HD) * T;
     g.err = err;
     const cudaError_t e = launch_gemm(xmap, wmap, g, static_cast<int>(ceil_div(HD, kBN)), 1, 1, st);
-    if (e != cudaSuccess) return SAGA_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_fail(e, "key GEMM");
   }
   // 3a. C partials: segments hi.hi, hi.lo, lo.hi over T
   {
@@ -603,7 +605,7 @@ extern "C" saga_status saga_merge_keys(const saga_merge_shape *shape, const void
     g.err = err;
     const cudaError_t e = launch_gemm(ktmap, ktmap, g, static_cast<int>(ceil_div(HD, kBN)),
                                       p.splits_c, 1, st);
-    if (e != cudaSuccess) return SAGA_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_fail(e, "key Gram GEMM");
   }
   // 3b. S partials: batch r, one segment per query head j = r*G + s; rows j*d ..
   {
@@ -622,7 +624,7 @@ extern "C" saga_status saga_merge_keys(const saga_merge_shape *shape, const void
     g.out_split = static_cast<long long>(s.h_k) * d * d;
     g.err = err;
     const cudaError_t e = launch_gemm(qtmap, qtmap, g, 1, p.splits_s, s.h_k, st);
-    if (e != cudaSuccess) return SAGA_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_fail(e, "query Gram GEMM");
   }
   // 4. float64 sums of the partials
   {
@@ -632,17 +634,17 @@ extern "C" saga_status saga_merge_keys(const saga_merge_shape *shape, const void
                        0, st>>>(C_part, nc, p.splits_c, nc, C_sum);
     km_reduce_kernel<<<static_cast<unsigned>(std::min<long long>(ceil_div(ns, 256), 4096)), 256,
                        0, st>>>(S_part, ns, p.splits_s, ns, S_sum);
-    if (cudaGetLastError() != cudaSuccess) return SAGA_ERR_CUDA;
+    if (const cudaError_t e = cudaGetLastError(); e != cudaSuccess) return cuda_fail(e, "reduce kernel");
   }
   // 5. per pair: pseudoinverse, A_a, A_b, w(a, b)
   {
     const cudaError_t e = d == 64 ? launch_pair<64, double>(S_sum, C_sum, s.h_k, rcond, Ag, w, st)
                                   : launch_pair<128, float>(S_sum, C_sum, s.h_k, rcond, Ag, w, st);
-    if (e != cudaSuccess) return SAGA_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_fail(e, "pair kernel");
   }
   // 6. the matching
   km_match_kernel<<<1, kMatchThreads, 0, st>>>(w, s.h_k, f, choice, pairs, total);
-  if (cudaGetLastError() != cudaSuccess) return SAGA_ERR_CUDA;
+  if (const cudaError_t e = cudaGetLastError(); e != cudaSuccess) return cuda_fail(e, "matching kernel");
   // 7. the student's key projection
   {
     const dim3 grid(static_cast<unsigned>(ceil_div(s.d_model, kProjX)),
@@ -653,7 +655,7 @@ extern "C" saga_status saga_merge_keys(const saga_merge_shape *shape, const void
     else
       km_project_kernel<128><<<grid, kProjX, 0, st>>>(static_cast<const uint16_t *>(W_K),
                                                      s.d_model, s.h_k, pairs, Ag, W_S);
-    if (cudaGetLastError() != cudaSuccess) return SAGA_ERR_CUDA;
+    if (const cudaError_t e = cudaGetLastError(); e != cudaSuccess) return cuda_fail(e, "projection kernel");
   }
   return SAGA_OK;
 }

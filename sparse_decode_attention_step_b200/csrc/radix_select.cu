@@ -8,7 +8,8 @@
 // the remaining rank. After four digits the prefix is the full key of an
 // element of the row, so tau is always one of the row's own scores.
 //
-// One CTA per row. Digit 0 comes from the histogram the score pass already
+// One CTA of 512 threads per row, two CTAs per SM, launched with programmatic
+// stream serialisation after the score pass. Digit 0 comes from the histogram the score pass already
 // built (or from one pass over the row). A second pass over the row fixes
 // digit 1 and copies the keys of the digit-0 bucket into shared memory; the
 // last two digits are found there. When that bucket does not fit (its scores
@@ -21,6 +22,8 @@
 // rank left inside tau's bucket is the number k of entries equal to tau that
 // the N largest include, and one more pass in position order finds the
 // position of the k-th of them.
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -28,13 +31,16 @@ namespace saga {
 
 namespace {
 
-constexpr int kThreads = 1024;
-constexpr int kCand = 32768;                        // candidate keys kept on chip (128 KB)
+constexpr int kThreads = 512;
+constexpr int kCtasPerSm = 2;                       // two rows streamed per SM at a time
+constexpr int kCand = 16384;                        // candidate keys kept on chip (64 KB)
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxDevices = 64;
 
 struct Shared {
   uint32_t hist[256];
   uint32_t digit, rem, n_cand;
-  uint32_t wsum[32];
+  uint32_t wsum[kWarps];
   int32_t found;
 };
 
@@ -80,19 +86,26 @@ __device__ __forceinline__ void pick_digit(Shared &sh, int lane) {
   }
 }
 
-// Visit every element t < L of a row as f(key, valid), all threads of the
-// CTA in step (f may use warp votes). Each thread keeps kVec * 4 elements in
-// flight per step (16-byte loads when the row is 16-byte aligned).
+// Visit a row in steps of kThreads * kVec * 4 elements, all threads of the
+// CTA in step: f(v, t0) gets this thread's kVec * 4 values, v[u][e] being
+// element elem_index(t0, tid, u, e); elements at or past L read as 0 and the
+// visitor checks the index against L. 16-byte loads when the row is 16-byte
+// aligned; kVec * 16 bytes in flight per thread.
 constexpr int kVec = 4;
+constexpr int64_t kStep = static_cast<int64_t>(kThreads) * kVec * 4;
+
+__device__ __forceinline__ int64_t elem_index(int64_t t0, int tid, int u, int e) {
+  return t0 + (static_cast<int64_t>(u) * kThreads + tid) * 4 + e;
+}
+
 template <typename F>
-__device__ __forceinline__ void for_row(const float *row, int64_t L, int tid, F f) {
-  constexpr int64_t kStep = static_cast<int64_t>(kThreads) * kVec * 4;
+__device__ __forceinline__ void for_row_steps(const float *row, int64_t L, int tid, F f) {
   const bool vec = (reinterpret_cast<uintptr_t>(row) & 15u) == 0;
   for (int64_t t0 = 0; t0 < L; t0 += kStep) {
     float v[kVec][4];
 #pragma unroll
     for (int u = 0; u < kVec; ++u) {
-      const int64_t i = t0 + (static_cast<int64_t>(u) * kThreads + tid) * 4;
+      const int64_t i = elem_index(t0, tid, u, 0);
       if (vec && i + 3 < L) {
         const float4 x = __ldg(reinterpret_cast<const float4 *>(row + i));
         v[u][0] = x.x; v[u][1] = x.y; v[u][2] = x.z; v[u][3] = x.w;
@@ -101,22 +114,71 @@ __device__ __forceinline__ void for_row(const float *row, int64_t L, int tid, F 
         for (int e = 0; e < 4; ++e) v[u][e] = i + e < L ? __ldg(row + i + e) : 0.f;
       }
     }
-#pragma unroll
-    for (int u = 0; u < kVec; ++u) {
-      const int64_t i = t0 + (static_cast<int64_t>(u) * kThreads + tid) * 4;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) f(order_key(v[u][e]), i + e < L);
-    }
+    f(v, t0);
   }
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+// Element-wise visit: f(key, valid) for every element of the row.
+template <typename F>
+__device__ __forceinline__ void for_row(const float *row, int64_t L, int tid, F f) {
+  for_row_steps(row, L, tid, [&](const float (&v)[kVec][4], int64_t t0) {
+#pragma unroll
+    for (int u = 0; u < kVec; ++u)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) f(order_key(v[u][e]), elem_index(t0, tid, u, e) < L);
+  });
+}
+
+// Copy the keys of the row with (key & mask) == prefix into cand (as many as
+// fit; the returned count may exceed kCand) and, when `shift` >= 0, count
+// digit `shift` of those keys into hist. One shared atomic per warp and step
+// reserves the warp's candidate slots.
+__device__ __forceinline__ void collect(const float *row, int64_t L, int tid, int lane,
+                                        uint32_t mask, uint32_t prefix, int shift, Shared &sh,
+                                        uint32_t *cand) {
+  for_row_steps(row, L, tid, [&](const float (&v)[kVec][4], int64_t t0) {
+    uint32_t c = 0;
+#pragma unroll
+    for (int u = 0; u < kVec; ++u)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        c += (elem_index(t0, tid, u, e) < L && (order_key(v[u][e]) & mask) == prefix) ? 1u : 0u;
+    uint32_t incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
+    if (total != 0u) {
+      uint32_t base = 0;
+      if (lane == 31) base = atomicAdd(&sh.n_cand, total);
+      uint32_t at = __shfl_sync(0xffffffffu, base, 31) + incl - c;
+#pragma unroll
+      for (int u = 0; u < kVec; ++u)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t k = order_key(v[u][e]);
+          const bool in = elem_index(t0, tid, u, e) < L && (k & mask) == prefix;
+          if (in) {
+            if (at < static_cast<uint32_t>(kCand)) cand[at] = k;
+            ++at;
+          }
+          if (shift >= 0) count_key(k, in, 0u, 0u, shift, sh.hist, lane);
+        }
+    }
+  });
+}
+
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
 radix_select_kernel(const float *__restrict__ scores, int64_t row_stride,
                     const int32_t *__restrict__ l_kv, int N, float *__restrict__ tau, int h_q,
                     int64_t cap, int64_t max_l_kv, const uint32_t *__restrict__ hist0,
                     int32_t *__restrict__ tie) {
   __shared__ Shared sh;
   extern __shared__ uint32_t cand[];
+  pdl_wait();
+  pdl_trigger();
   const int bj = blockIdx.x;
   const int b = bj / h_q;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -154,20 +216,7 @@ radix_select_kernel(const float *__restrict__ scores, int64_t row_stride,
   // ---- digit 1: one pass over the row; keep the digit-0 bucket on chip -----
   for (int i = tid; i < 256; i += kThreads) sh.hist[i] = 0u;
   __syncthreads();
-  for_row(row, L, tid, [&](uint32_t k, bool valid) {
-    const bool in = valid && (k & mask) == prefix;
-    const uint32_t bal = __ballot_sync(0xffffffffu, in);
-    if (bal != 0u) {
-      uint32_t base = 0;
-      if (lane == 0) base = atomicAdd(&sh.n_cand, static_cast<uint32_t>(__popc(bal)));
-      base = __shfl_sync(0xffffffffu, base, 0);
-      if (in) {
-        const uint32_t at = base + __popc(bal & ((1u << lane) - 1u));
-        if (at < static_cast<uint32_t>(kCand)) cand[at] = k;
-      }
-    }
-    count_key(k, valid, mask, prefix, 16, sh.hist, lane);
-  });
+  collect(row, L, tid, lane, mask, prefix, 16, sh, cand);
   __syncthreads();
   if (warp == 0) pick_digit(sh, lane);
   __syncthreads();
@@ -181,19 +230,7 @@ radix_select_kernel(const float *__restrict__ scores, int64_t row_stride,
     // the 16-bit prefix instead, with one more pass over the row
     if (tid == 0) sh.n_cand = 0;
     __syncthreads();
-    for_row(row, L, tid, [&](uint32_t k, bool valid) {
-      const bool in = valid && (k & mask) == prefix;
-      const uint32_t bal = __ballot_sync(0xffffffffu, in);
-      if (bal != 0u) {
-        uint32_t base = 0;
-        if (lane == 0) base = atomicAdd(&sh.n_cand, static_cast<uint32_t>(__popc(bal)));
-        base = __shfl_sync(0xffffffffu, base, 0);
-        if (in) {
-          const uint32_t at = base + __popc(bal & ((1u << lane) - 1u));
-          if (at < static_cast<uint32_t>(kCand)) cand[at] = k;
-        }
-      }
-    });
+    collect(row, L, tid, lane, mask, prefix, -1, sh, cand);
     __syncthreads();
     n_cand = sh.n_cand;
     on_chip = n_cand <= static_cast<uint32_t>(kCand);
@@ -248,13 +285,13 @@ radix_select_kernel(const float *__restrict__ scores, int64_t row_stride,
     if (lane == 31) sh.wsum[warp] = incl;
     __syncthreads();
     if (warp == 0) {
-      uint32_t ws = sh.wsum[lane];
+      uint32_t ws = lane < kWarps ? sh.wsum[lane] : 0u;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const uint32_t y = __shfl_up_sync(0xffffffffu, ws, o);
         if (lane >= o) ws += y;
       }
-      sh.wsum[lane] = ws;                       // inclusive over warps
+      if (lane < kWarps) sh.wsum[lane] = ws;    // inclusive over warps
     }
     __syncthreads();
     const uint32_t excl = before + (warp > 0 ? sh.wsum[warp - 1] : 0u) + (incl - c);
@@ -263,7 +300,7 @@ radix_select_kernel(const float *__restrict__ scores, int64_t row_stride,
       while (--need) hh &= hh - 1u;
       sh.found = static_cast<int32_t>(i + __ffs(hh) - 1);
     }
-    before += sh.wsum[kThreads / 32 - 1];
+    before += sh.wsum[kWarps - 1];
     __syncthreads();
     if (sh.found >= 0) break;
   }
@@ -275,17 +312,21 @@ radix_select_kernel(const float *__restrict__ scores, int64_t row_stride,
 cudaError_t launch_radix_select(const float *scores, int64_t row_stride, const int32_t *l_kv,
                                 int N, float *tau, int B, int h_q, int64_t cap, int64_t max_l_kv,
                                 const uint32_t *hist0, int32_t *tie, cudaStream_t st) {
-  static bool attr_set = false;
+  // the dynamic shared-memory opt-in is per device; set once on each
+  static std::atomic<bool> attr_set[kMaxDevices];
   const int smem = kCand * static_cast<int>(sizeof(uint32_t));
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(radix_select_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (!attr_set[dev].load(std::memory_order_acquire)) {
+    e = cudaFuncSetAttribute(radix_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
-  radix_select_kernel<<<B * h_q, kThreads, smem, st>>>(scores, row_stride, l_kv, N, tau, h_q,
-                                                       cap, max_l_kv, hist0, tie);
-  return cudaGetLastError();
+  return launch_pdl(radix_select_kernel, dim3(B * h_q), dim3(kThreads), smem, st, scores,
+                    row_stride, l_kv, N, tau, h_q, cap, max_l_kv, hist0, tie);
 }
 
 }  // namespace saga

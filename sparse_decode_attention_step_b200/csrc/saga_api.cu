@@ -3,6 +3,7 @@
 // Nothing here allocates device memory or synchronises, except
 // saga_read_device_error, which synchronises by contract.
 #include <cmath>
+#include <cstdio>
 #include <cstring>
 
 #include "common.cuh"
@@ -128,7 +129,6 @@ StepParams base_params(const saga_shape &s, const Plan &pl, const void *q, const
 
 int group_pad(const saga_shape &s) { return ((s.h_q / s.h_k) + 3) / 4 * 4; }
 
-saga_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SAGA_OK : SAGA_ERR_CUDA; }
 
 // The tensor-core kernel takes the score-producing modes (dump, step) of the
 // shapes it supports (a failure there is reported, never replaced by another
@@ -148,10 +148,10 @@ cudaError_t launch_split(const saga_shape &s, const StepParams &p, int mode, cud
 saga_status run_step(const saga_shape &s, const Plan &pl, StepParams p, int mode,
                      float *out, int32_t *sel_count, cudaStream_t st) {
   cudaError_t e = launch_split(s, p, mode, st);
-  if (e != cudaSuccess) return SAGA_ERR_CUDA;
-  e = launch_combine(p.partials, p.l_kv, p.err, out, sel_count, s.B, s.h_q, s.d, pl.S,
-                     pl.split_len, s.cap, s.max_l_kv, st);
-  return cuda_status(e);
+  if (e != cudaSuccess) return cuda_fail(e, p.scores_in ? "step kernel (stored scores)" : "step kernel");
+  return cuda_check(launch_combine(p.partials, p.l_kv, p.err, out, sel_count, s.B, s.h_q, s.d,
+                                   pl.S, pl.split_len, s.cap, s.max_l_kv, st),
+                    "combine kernel");
 }
 
 // Full attention (Eq. 2-4) with the shape's key and value head maps: the
@@ -168,13 +168,22 @@ saga_status run_dense(const saga_shape &s, const void *q, const void *K, const v
   const Plan pl = make_plan(s, false, dense_ctas_per_sm(s.dtype, s.d, s.h_q, s.h_k, s.h_v));
   StepParams p = base_params(s, pl, q, K, V, l_kv, ws);
   cudaError_t e = launch_dense_split(p, s.dtype, s.d, st);
-  if (e != cudaSuccess) return SAGA_ERR_CUDA;
-  e = launch_combine(p.partials, l_kv, p.err, out, nullptr, s.B, s.h_q, s.d, pl.S, pl.split_len,
-                     s.cap, s.max_l_kv, st);
-  return cuda_status(e);
+  if (e != cudaSuccess) return cuda_fail(e, "dense kernel");
+  return cuda_check(launch_combine(p.partials, l_kv, p.err, out, nullptr, s.B, s.h_q, s.d, pl.S,
+                                   pl.split_len, s.cap, s.max_l_kv, st),
+                    "combine kernel");
 }
 
+thread_local char g_last_error[256] = "";
+
 }  // namespace
+
+saga_status cuda_fail(cudaError_t e, const char *where) {
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%s)", where, cudaGetErrorName(e),
+                cudaGetErrorString(e));
+  cudaGetLastError();   // a failed launch's error is not sticky: clear it for the next call
+  return SAGA_ERR_CUDA;
+}
 
 // Scratch a plain step needs (error word + per-split states; no score rows).
 size_t plain_step_scratch_bytes(const saga_shape &s) { return saga_plan(s).off_scores; }
@@ -225,7 +234,8 @@ size_t saga_workspace_size(const saga_shape *shape, int32_t N) {
 
 saga_status saga_workspace_init(void *ws, size_t ws_bytes, saga_stream_t stream) {
   if (ws == nullptr || !aligned(ws, kAlign) || ws_bytes < kAlign) return SAGA_ERR_WORKSPACE;
-  return cuda_status(cudaMemsetAsync(ws, 0, kAlign, reinterpret_cast<cudaStream_t>(stream)));
+  return cuda_check(cudaMemsetAsync(ws, 0, kAlign, reinterpret_cast<cudaStream_t>(stream)),
+                    "cudaMemsetAsync (error word)");
 }
 
 saga_status saga_decode_step(const saga_shape *shape, const void *q, const void *K,
@@ -272,27 +282,32 @@ saga_status saga_refresh_threshold(const saga_shape *shape, const void *q, const
   uint32_t *hist = nullptr;
   if (use_tc(s)) {
     hist = reinterpret_cast<uint32_t *>(static_cast<char *>(ws) + pl.off_hist);
-    if (cudaMemsetAsync(hist, 0, static_cast<size_t>(s.B) * s.h_q * 256 * sizeof(uint32_t), st) !=
-        cudaSuccess)
-      return SAGA_ERR_CUDA;
+    const cudaError_t me =
+        cudaMemsetAsync(hist, 0, static_cast<size_t>(s.B) * s.h_q * 256 * sizeof(uint32_t), st);
+    if (me != cudaSuccess) return cuda_fail(me, "cudaMemsetAsync (histograms)");
   }
   p.scores_out = rows;
   p.hist = hist;
   cudaError_t e = launch_split(s, p, kModeDump, st);
-  if (e != cudaSuccess) return SAGA_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_fail(e, "score dump kernel");
   // 2. exact N-th largest per row
   e = launch_radix_select(rows, s.max_l_kv, l_kv, N, tau, s.B, s.h_q, s.cap, s.max_l_kv, hist,
                           nullptr, st);
-  if (e != cudaSuccess) return SAGA_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_fail(e, "radix select kernel");
   if (V == nullptr) return SAGA_OK;
-  // 3. this step's select + PV with the fresh tau. Tensor-core shapes: the
-  // step kernel recomputes the scores with the same MMAs, so they equal the
-  // rows tau came from bit for bit; other shapes read the stored rows back.
+  // 3. this step's select + PV with the fresh tau, over the very rows tau
+  // came from: streamed back from memory (K is not read again), or, on the
+  // tensor-core path when the rows cannot be streamed (a caller's buffer
+  // with an odd stride), recomputed from K with the same MMAs, which gives
+  // the same scores bit for bit.
   p.scores_out = nullptr;
   p.hist = nullptr;
   p.tau = tau;
   p.sel_mask = sel_mask;
-  if (use_tc(s)) return run_step(s, pl, p, kModeStep, out, sel_count, st);
+  if (use_tc(s)) {
+    if (saga_tc_scores_streamable(rows, s.max_l_kv)) p.scores_in = rows;
+    return run_step(s, pl, p, kModeStep, out, sel_count, st);
+  }
   p.scores_in = rows;
   return run_step(s, pl, p, kModeFromScores, out, sel_count, st);
 }
@@ -321,26 +336,30 @@ saga_status saga_topn_step(const saga_shape *shape, const void *q, const void *K
   uint32_t *hist = nullptr;
   if (use_tc(s)) {
     hist = reinterpret_cast<uint32_t *>(wsb + pl.off_hist);
-    if (cudaMemsetAsync(hist, 0, static_cast<size_t>(s.B) * s.h_q * 256 * sizeof(uint32_t), st) !=
-        cudaSuccess)
-      return SAGA_ERR_CUDA;
+    const cudaError_t me =
+        cudaMemsetAsync(hist, 0, static_cast<size_t>(s.B) * s.h_q * 256 * sizeof(uint32_t), st);
+    if (me != cudaSuccess) return cuda_fail(me, "cudaMemsetAsync (histograms)");
   }
   p.scores_out = rows;
   p.hist = hist;
   cudaError_t e = launch_split(s, p, kModeDump, st);
-  if (e != cudaSuccess) return SAGA_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_fail(e, "score dump kernel");
   // 2. the N-th largest and, when it is tied, the last tied position taken
   e = launch_radix_select(rows, s.max_l_kv, l_kv, N, tau, s.B, s.h_q, s.cap, s.max_l_kv, hist,
                           tie, st);
-  if (e != cudaSuccess) return SAGA_ERR_CUDA;
-  // 3. the step over exactly those positions (bit-identical scores again on
-  // the tensor-core path, the stored rows otherwise)
+  if (e != cudaSuccess) return cuda_fail(e, "radix select kernel");
+  // 3. the step over exactly those positions, from the stored rows (or, on
+  // the tensor-core path when they cannot be streamed, from bit-identical
+  // scores recomputed from K)
   p.scores_out = nullptr;
   p.hist = nullptr;
   p.tau = tau;
   p.tie = tie;
   p.sel_mask = sel_mask;
-  if (use_tc(s)) return run_step(s, pl, p, kModeStepTies, out, sel_count, st);
+  if (use_tc(s)) {
+    if (saga_tc_scores_streamable(rows, s.max_l_kv)) p.scores_in = rows;
+    return run_step(s, pl, p, kModeStepTies, out, sel_count, st);
+  }
   p.scores_in = rows;
   return run_step(s, pl, p, kModeFromScores, out, sel_count, st);
 }
@@ -375,9 +394,10 @@ saga_status saga_append_kv(const saga_shape *shape, const void *k_new, const voi
     return SAGA_ERR_INVALID_ARG;
   if (ws == nullptr || !aligned(ws, kAlign) || ws_bytes < kAlign) return SAGA_ERR_WORKSPACE;
   const int esz = s.dtype == SAGA_F32 ? 4 : 2;
-  return cuda_status(launch_append(k_new, v_new, K, V, l_kv, static_cast<int32_t *>(ws), s.B, s.h_k,
+  return cuda_check(launch_append(k_new, v_new, K, V, l_kv, static_cast<int32_t *>(ws), s.B, s.h_k,
                                    s.h_v, s.d, esz, s.k_stride_b, s.k_stride_h, s.v_stride_b,
-                                   s.v_stride_h, s.cap, reinterpret_cast<cudaStream_t>(stream)));
+                                   s.v_stride_h, s.cap, reinterpret_cast<cudaStream_t>(stream)),
+                    "append kernel");
 }
 
 saga_status saga_debug_scores(const saga_shape *shape, const void *q, const void *K,
@@ -393,20 +413,24 @@ saga_status saga_debug_scores(const saga_shape *shape, const void *q, const void
   StepParams p = base_params(s, pl, q, K, nullptr, l_kv, ws);
   p.partials = nullptr;
   p.scores_out = scores;
-  return cuda_status(launch_split(s, p, kModeDump, reinterpret_cast<cudaStream_t>(stream)));
+  return cuda_check(launch_split(s, p, kModeDump, reinterpret_cast<cudaStream_t>(stream)),
+                    "score dump kernel");
 }
 
 saga_status saga_read_device_error(void *ws, saga_stream_t stream, int32_t *flags) {
   if (ws == nullptr || !aligned(ws, kAlign) || flags == nullptr) return SAGA_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   int32_t h = 0;
-  if (cudaMemcpyAsync(&h, ws, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess)
-    return SAGA_ERR_CUDA;
-  if (cudaMemsetAsync(ws, 0, sizeof(int32_t), st) != cudaSuccess) return SAGA_ERR_CUDA;
-  if (cudaStreamSynchronize(st) != cudaSuccess) return SAGA_ERR_CUDA;
+  cudaError_t e = cudaMemcpyAsync(&h, ws, sizeof(h), cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync (error word)");
+  if ((e = cudaMemsetAsync(ws, 0, sizeof(int32_t), st)) != cudaSuccess)
+    return cuda_fail(e, "cudaMemsetAsync (error word)");
+  if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
   *flags = h;
   return h != 0 ? SAGA_ERR_DEVICE : SAGA_OK;
 }
+
+const char *saga_last_error(void) { return g_last_error; }
 
 const char *saga_status_string(saga_status status) {
   switch (status) {

@@ -31,11 +31,15 @@ void *g_ptr[kMaxDevices] = {};
 // device (host code cannot use the symbol itself as a device pointer).
 saga_status scratch_for_current_device(void **out) {
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SAGA_ERR_CUDA;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return saga::cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return saga::cuda_fail(cudaErrorInvalidDevice, "device index");
   std::lock_guard<std::mutex> lock(g_mu);
   if (g_ptr[dev] == nullptr) {
     void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || p == nullptr) return SAGA_ERR_CUDA;
+    e = cudaGetSymbolAddress(&p, g_scratch);
+    if (e != cudaSuccess) return saga::cuda_fail(e, "cudaGetSymbolAddress (no-alloc scratch)");
+    if (p == nullptr) return saga::cuda_fail(cudaErrorInvalidSymbol, "cudaGetSymbolAddress (no-alloc scratch)");
     g_ptr[dev] = p;
   }
   *out = g_ptr[dev];

@@ -16,28 +16,35 @@
 //   workers     4 x kRanks warps. Tile g belongs to rank g % kRanks; each of
 //               the four warps of that rank reads its TMEM lane quarter
 //               (32 keys x 16 heads), scales by 1/sqrt(d), compares with tau
-//               and then gathers V for its own kept keys: lane group v (8
-//               lanes) owns up to four query heads that share one value
-//               head, so each kept V row is read once for all of them, and
-//               keeps their online-softmax states in registers (rows in
-//               batches of kRows; empty rows and heads no lane group kept are
-//               skipped, and the states are rescaled only when a batch raises
-//               a maximum). At the end of a unit every worker writes its states
-//               to shared memory, the per-head weights e^{m_w - m} are formed
-//               once, and all workers write the unit's (m, l, count, acc)
-//               records.
+//               and gathers V for its own kept keys: lane group v (8 lanes)
+//               owns up to four query heads that share one value head, so
+//               each kept V row is read once for all of them, and keeps their
+//               online-softmax states (m, l, count, acc) in registers.
+//
+// Each worker folds a quarter tile's kept rows in rounds of kRows V rows per
+// lane group (empty rows and heads no lane group kept are skipped, and the
+// states are rescaled only when a round raises a maximum). At the end of a
+// unit every worker writes its states to shared memory, the per-head
+// weights e^{m_w - m} are formed once, and all workers write the unit's
+// (m, l, count, acc) records.
 //
 // Modes: dump (score rows and per-row top-byte histograms of the order keys,
 // for a refresh), step (keep A >= tau), step with ties (exact top-N: keep A
-// above tau under totalOrder, and A == tau up to a per-row position).
+// above tau under totalOrder, and A == tau up to a per-row position). The
+// step modes also run from stored score rows (FS): the producer then streams
+// [16 heads x 128 positions] fp32 tiles of the refresh's own rows instead of
+// K and no MMA runs, so a refresh reads K only once.
 //
 // Query heads beyond the group (G < 16) are rows of other heads or zero rows
 // of Q; their tau is +inf, so they are never kept, and they are never dumped.
-// Every wait is bounded; on a timeout the CTA sets SAGA_DEVERR_TIMEOUT and
-// all roles stop, after the copies and MMAs in flight have landed.
+// Every wait is bounded; on a timeout the CTA sets SAGA_DEVERR_TIMEOUT, all
+// roles stop after the copies and MMAs in flight have landed, and the
+// workers write poisoned records (m = +inf, count = -1) for every unit the
+// CTA had left, which the combine turns into NaN outputs and counts of -1.
 #include <cuda.h>
 
 #include <atomic>
+#include <cstring>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -49,7 +56,6 @@ namespace {
 
 constexpr int kTileKeys = 128;
 constexpr int kN = 16;                      // MMA N: query heads of a group, padded
-constexpr int kRows = 4;                    // kept V rows in flight per lane group
 constexpr int kWorkerBar = 1;               // named barrier of the worker warps
 constexpr uint32_t kIdesc = sm100::idesc_bf16_f32(kTileKeys, kN);
 constexpr float kLog2e = 1.4426950408889634f;
@@ -70,6 +76,9 @@ struct Cfg {
   static constexpr int kTileBytes = kBoxes * kBoxBytes;
   static constexpr int kQBoxBytes = kN * 128;
   static constexpr int kQBytes = kBoxes * kQBoxBytes;
+  static constexpr int kRows = 4;                              // kept V rows in flight per lane group
+  static constexpr int kScoreTileBytes = kN * kTileKeys * 4;   // FS stage: [16][128] fp32
+  static_assert(kScoreTileBytes <= kTileBytes, "a score tile fits a stage");
   static constexpr int CPL = D / 64;                           // 16-byte chunks per lane per V row
   static constexpr int EPL = 8 * CPL;                          // V row elements per lane
   static constexpr int kRec = D + kRecPad;
@@ -220,13 +229,23 @@ __device__ __forceinline__ void put_state(float *r, int c8, float m, float l, in
   }
 }
 
-template <int D, int MODE>
+// Poisoned record: the combine turns it into a NaN output and a count of -1.
+__device__ __forceinline__ void put_poison(float *r) {
+  r[0] = INFINITY;
+  r[1] = __int_as_float(0x7fc00000);
+  r[2] = __int_as_float(-1);
+  r[3] = 0.f;
+}
+
+template <int D, int MODE, bool FS>
 __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
 saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
                const __grid_constant__ CUtensorMap qmap, const HeadMap hm) {
   using C = Cfg<D>;
   using Lo = Layout<D>;
-  constexpr int CPL = C::CPL, EPL = C::EPL;
+  constexpr int CPL = C::CPL, EPL = C::EPL, kRows = C::kRows;
+  constexpr bool kDump = MODE == kModeDump;
+  static_assert(!(kDump && FS), "the dump reads K");
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = sm100::smem_u32(smem_raw);
@@ -241,11 +260,11 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
   const int vpg = p.h_v / p.h_k;
   const int n_units = p.B * p.h_k * p.S;
 
-  // ---- set-up --------------------------------------------------------------
+  // ---- set-up (touches no global memory) ---------------------------------
   if (tid == 0) {
     for (int i = 0; i < C::kStages; ++i) {
       sm100::mbar_init(&h->full[i], 1);
-      sm100::mbar_init(&h->empty[i], 1);
+      sm100::mbar_init(&h->empty[i], FS ? 4 : 1);   // FS: the rank's four warps free a stage
     }
     for (int i = 0; i < C::kTBufs; ++i) {
       sm100::mbar_init(&h->tfull[i], 1);
@@ -258,54 +277,65 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
     h->abort = 0;
     sm100::fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == 1 && !FS) {
     sm100::tmem_alloc(&h->tmem_base, C::kTmemCols);
     sm100::tmem_relinquish();
   }
-  if (MODE == kModeDump && p.hist != nullptr && warp >= 2) {
+  if (kDump && p.hist != nullptr && warp >= 2) {
     uint32_t *hs = reinterpret_cast<uint32_t *>(scratch);
     for (int i = tid - 64; i < kN * 256; i += C::kWorkers * 32) hs[i] = 0u;
   }
   sm100::tc_fence_before();
   __syncthreads();
   sm100::tc_fence_after();
-  const uint32_t tmem_base = h->tmem_base;
+  const uint32_t tmem_base = FS ? 0u : h->tmem_base;
+  // everything below may read what the previous launch in the stream wrote
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 0) {
     // ---- TMA producer ------------------------------------------------------
     if (lane == 0) {
       sm100::prefetch_tensormap(&kmap);
-      sm100::prefetch_tensormap(&qmap);
+      if (!FS) sm100::prefetch_tensormap(&qmap);
       uint32_t g = 0;
       int k = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
         Unit un;
         if (!unit_at(p, u, true, un)) continue;
-        const int qb = k & 1;
-        if (!wait_bar(&h->qempty[qb], ((k >> 1) & 1) ^ 1, h)) { ok = false; break; }
-        sm100::mbar_arrive_expect_tx(&h->qfull[qb], C::kQBytes);
+        if (!FS) {
+          const int qb = k & 1;
+          if (!wait_bar(&h->qempty[qb], ((k >> 1) & 1) ^ 1, h)) { ok = false; break; }
+          sm100::mbar_arrive_expect_tx(&h->qfull[qb], C::kQBytes);
 #pragma unroll
-        for (int bx = 0; bx < C::kBoxes; ++bx)
-          sm100::tma_load_3d(qbuf + qb * C::kQBytes + bx * C::kQBoxBytes, &qmap, &h->qfull[qb],
-                             bx * 64, un.kh * G, un.b);
-        ++k;
+          for (int bx = 0; bx < C::kBoxes; ++bx)
+            sm100::tma_load_3d(qbuf + qb * C::kQBytes + bx * C::kQBoxBytes, &qmap, &h->qfull[qb],
+                               bx * 64, un.kh * G, un.b);
+          ++k;
+        }
         for (int i = 0; i < un.n_tiles; ++i) {
           const int st = g % C::kStages;
           if (!wait_bar(&h->empty[st], ((g / C::kStages) & 1) ^ 1, h)) { ok = false; break; }
-          sm100::mbar_arrive_expect_tx(&h->full[st], C::kTileBytes);
           const int y = static_cast<int>(un.t_begin) + i * kTileKeys;
+          uint8_t *dst = stages + st * C::kTileBytes;
+          if (FS) {
+            sm100::mbar_arrive_expect_tx(&h->full[st], C::kScoreTileBytes);
+            sm100::tma_load_3d(dst, &kmap, &h->full[st], y, un.kh * G, un.b);
+          } else {
+            sm100::mbar_arrive_expect_tx(&h->full[st], C::kTileBytes);
 #pragma unroll
-          for (int bx = 0; bx < C::kBoxes; ++bx)
-            sm100::tma_load_4d(stages + st * C::kTileBytes + bx * C::kBoxBytes, &kmap,
-                               &h->full[st], bx * 64, y, un.kh, un.b);
+            for (int bx = 0; bx < C::kBoxes; ++bx)
+              sm100::tma_load_4d(dst + bx * C::kBoxBytes, &kmap, &h->full[st], bx * 64, y, un.kh,
+                                 un.b);
+          }
           ++g;
         }
       }
       if (!ok) {
         fail(p, h);
         // the copies still in flight land before the CTA can exit: the
-        // last kStages K tiles and the last two Q tiles
+        // last kStages tiles and the last two Q tiles
         for (uint32_t i = g > static_cast<uint32_t>(C::kStages) ? g - C::kStages : 0; i < g; ++i)
           sm100::mbar_wait(&h->full[i % C::kStages], (i / C::kStages) & 1);
         for (int i = k > 2 ? k - 2 : 0; i < k; ++i)
@@ -314,8 +344,8 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---- MMA issuer ----------------------------------------------------------
-    if (lane == 0) {
+    // ---- MMA issuer (idle when the scores come from stored rows) ------------
+    if (lane == 0 && !FS) {
       const uint32_t st_u32 = sm100::smem_u32(stages);
       const uint32_t q_u32 = sm100::smem_u32(qbuf);
       uint32_t g = 0, committed = 0;
@@ -364,12 +394,12 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
   } else {
     // ---- workers ------------------------------------------------------------
     const int widx = warp - 2;
-    const int quarter = warp & 3;             // TMEM lanes this warp may read
+    const int quarter = warp & 3;             // TMEM lanes (keys) this warp reads
     const int rank = widx >> 2;
     const int v = lane >> 3, c8 = lane & 7;
     const int hbase = pick4(hm.hbase, v), nh = pick4(hm.nh, v), vsl = pick4(hm.vs, v);
     const bool quad = (hbase & 3) == 0 && nh == 4;   // the heads are one 16-byte quad of a row
-    // two kept-score row sets, used in turn
+    // two kept-score row sets, used in turn: the rows in flight keep theirs
     float *rows_base = scratch + widx * 2 * 32 * kN;
     uint32_t g = 0;
     bool bad = false;
@@ -377,7 +407,6 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
     float m[4], l[4], acc[4][EPL];
     int cnt[4];
     const uint16_t *vrow = nullptr;
-
     // Fold the kept keys `mine` of this lane group (keys t0 + bit) into the
     // lane group's online-softmax states, kRows V rows in flight per round.
     auto gather = [&](uint32_t mine, int64_t t0, int64_t t_any, const float *rows) {
@@ -464,12 +493,13 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
       }
     };
 
-    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+    int u = blockIdx.x;
+    for (; u < n_units; u += gridDim.x) {
       Unit un;
       if (!unit_at(p, u, false, un)) continue;
       const int j0 = un.kh * G;
       const int64_t row0 = static_cast<int64_t>(un.b * p.h_q + j0) * p.row_stride;
-      if (MODE != kModeDump) {
+      if (!kDump) {
         if (widx == 0 && lane < kN) {
           h->tau[lane] = lane < G ? p.tau[un.b * p.h_q + j0 + lane] : INFINITY;
           if (MODE == kModeStepTies) h->tie[lane] = lane < G ? p.tie[un.b * p.h_q + j0 + lane] : -1;
@@ -489,24 +519,37 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
       const int first = (rank - static_cast<int>(g % C::kRanks) + C::kRanks) % C::kRanks;
       for (int i = first; i < un.n_tiles; i += C::kRanks) {
         const uint32_t gg = g + i;
-        const int tb = gg % C::kTBufs;
-        if (!warp_wait_bar(&h->tfull[tb], (gg / C::kTBufs) & 1, h)) {
-          if (lane == 0) fail(p, h);
-          bad = true;
-          break;
-        }
-        sm100::tc_fence_after();
         float A[kN];
-        sm100::tmem_ld16(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + tb * kN, A);
-        sm100::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) sm100::mbar_arrive(&h->tempty[tb]);
+        if (FS) {
+          const int st = gg % C::kStages;
+          if (!warp_wait_bar(&h->full[st], (gg / C::kStages) & 1, h)) {
+            if (lane == 0) fail(p, h);
+            bad = true;
+            break;
+          }
+          const float *sp = reinterpret_cast<const float *>(stages + st * C::kTileBytes);
+#pragma unroll
+          for (int a = 0; a < kN; ++a) A[a] = sp[a * kTileKeys + quarter * 32 + lane];
+          // the stage is freed below, once every lane has used its scores
+        } else {
+          const int tb = gg % C::kTBufs;
+          if (!warp_wait_bar(&h->tfull[tb], (gg / C::kTBufs) & 1, h)) {
+            if (lane == 0) fail(p, h);
+            bad = true;
+            break;
+          }
+          sm100::tc_fence_after();
+          sm100::tmem_ld16(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + tb * kN, A);
+          sm100::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) sm100::mbar_arrive(&h->tempty[tb]);
+        }
 
         const int64_t t0 = un.t_begin + static_cast<int64_t>(i) * kTileKeys + quarter * 32;
         const int64_t t = t0 + lane;
         const bool valid = t < un.t_end;
 
-        if (MODE == kModeDump) {
+        if (kDump) {
 #pragma unroll
           for (int a = 0; a < kN; ++a) {
             const float x = A[a] * p.scale;
@@ -541,7 +584,7 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int a = 4 * a4 + e;
-              const float x = A[a] * p.scale;
+              const float x = FS ? A[a] : A[a] * p.scale;
               bool keep;
               if constexpr (MODE == kModeStepTies) {
                 // totalOrder, as the threshold was selected: above tau, or
@@ -572,6 +615,9 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
           const uint32_t bl = __ballot_sync(0xffffffffu, (sel & hm.smask[vv]) != 0u);
           if (v == vv) mine = bl;
         }
+        // FS: every lane's scores have gone into `sel` and the ballots above,
+        // so the stage can be refilled
+        if (FS && lane == 0) sm100::mbar_arrive(&h->empty[gg % C::kStages]);
         __syncwarp();
         gather(mine, t0, un.t_begin, rows);
         __syncwarp();            // rows read before a later tile overwrites them
@@ -580,7 +626,7 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
 
       // ---- end of unit -------------------------------------------------------
       if (workers_any<D>(bad || aborted(h))) { bad = true; break; }
-      if (MODE == kModeDump) {
+      if (kDump) {
         if (p.hist != nullptr) {
           uint32_t *hs = reinterpret_cast<uint32_t *>(scratch);
           for (int i = widx * 32 + lane; i < kN * 256; i += C::kWorkers * 32) {
@@ -639,12 +685,21 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
       }
       workers_sync<D>();          // scratch read before the next unit reuses it
     }
+    if (bad && !kDump && widx == 0 && lane < kN) {
+      // this unit and every later one of this CTA: poisoned records
+      for (; u < n_units; u += gridDim.x) {
+        Unit un;
+        if (!unit_at(p, u, false, un) || lane >= G) continue;
+        const int j = un.kh * G + lane;
+        put_poison(p.partials + (static_cast<int64_t>(un.b * p.h_q + j) * p.S + un.s) * C::kRec);
+      }
+    }
   }
 
   // ---- teardown: every MMA has landed before TMEM is freed -----------------
   sm100::tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 1 && !FS) {
     sm100::tc_fence_after();
     sm100::tmem_dealloc(tmem_base, C::kTmemCols);
   }
@@ -685,13 +740,13 @@ int sm_count(int dev) {
   return n;
 }
 
-template <int D, int MODE>
+template <int D, int MODE, bool FS>
 cudaError_t launch_tc(const StepParams &p, const CUtensorMap &kmap, const CUtensorMap &qmap,
                       const HeadMap &hm, int dev, cudaStream_t st) {
   using Lo = Layout<D>;
   static std::atomic<bool> attr_set[kMaxDevices];
   if (!attr_set[dev].load(std::memory_order_acquire)) {
-    cudaError_t e = cudaFuncSetAttribute(saga_tc_kernel<D, MODE>,
+    cudaError_t e = cudaFuncSetAttribute(saga_tc_kernel<D, MODE, FS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Lo::alloc);
     if (e != cudaSuccess) return e;
     attr_set[dev].store(true, std::memory_order_release);
@@ -701,12 +756,12 @@ cudaError_t launch_tc(const StepParams &p, const CUtensorMap &kmap, const CUtens
   const int n_units = p.B * p.h_k * p.S;
   const int grid = n_units < sms ? n_units : sms;
   if (grid < 1) return cudaSuccess;
-  saga_tc_kernel<D, MODE><<<grid, Cfg<D>::kThreads, Lo::alloc, st>>>(p, kmap, qmap, hm);
-  return cudaGetLastError();
+  return launch_pdl(saga_tc_kernel<D, MODE, FS>, dim3(grid), dim3(Cfg<D>::kThreads), Lo::alloc,
+                    st, p, kmap, qmap, hm);
 }
 
-// Lane groups: value head slot vs = v / chunks, chunk c = v % chunks of that
-// value head's h_q / h_v query heads (four per chunk).
+// Lane-group slots: value head slot vs = v / chunks, chunk c = v % chunks of
+// that value head's h_q / h_v query heads (four per chunk).
 bool make_head_map(int h_q, int h_k, int h_v, HeadMap &hm) {
   if (h_k < 1 || h_v < 1 || h_q % h_v != 0 || h_v % h_k != 0) return false;
   const int G = h_q / h_k, hpv = h_q / h_v, vpg = h_v / h_k;
@@ -735,10 +790,18 @@ bool saga_tc_supports(int dtype, int d, int h_q, int h_k, int h_v) {
   return dtype == SAGA_BF16 && (d == 64 || d == 128) && make_head_map(h_q, h_k, h_v, hm);
 }
 
+bool saga_tc_scores_streamable(const float *rows, int64_t row_stride) {
+  return rows != nullptr && (reinterpret_cast<uintptr_t>(rows) % 16) == 0 && row_stride % 4 == 0 &&
+         row_stride > 0;
+}
+
 cudaError_t launch_saga_tc(const StepParams &p, int mode, int d, cudaStream_t st) {
   HeadMap hm;
   if (!make_head_map(p.h_q, p.h_k, p.h_v, hm)) return cudaErrorInvalidValue;
   if (mode != kModeDump && mode != kModeStep && mode != kModeStepTies) return cudaErrorInvalidValue;
+  const bool fs = p.scores_in != nullptr;
+  if (fs && (mode == kModeDump || !saga_tc_scores_streamable(p.scores_in, p.row_stride)))
+    return cudaErrorInvalidValue;
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return cudaErrorNotSupported;
   int dev = 0;
@@ -747,39 +810,55 @@ cudaError_t launch_saga_tc(const StepParams &p, int mode, int d, cudaStream_t st
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   CUtensorMap kmap, qmap;
-  {
-    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(p.cap),
-                                static_cast<cuuint64_t>(p.h_k), static_cast<cuuint64_t>(p.B)};
-    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2,
-                                   static_cast<cuuint64_t>(p.k_sh) * 2,
-                                   static_cast<cuuint64_t>(p.k_sb) * 2};
-    const cuuint32_t box[4] = {64, kTileKeys, 1, 1};
-    if (enc(&kmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(p.K), dims, strides,
-            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  std::memset(&qmap, 0, sizeof(qmap));
+  if (fs) {
+    // stored score rows [B][h_q][row_stride] fp32: a [16 heads x 128 positions] box
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(p.max_l_kv), static_cast<cuuint64_t>(p.h_q),
+                                static_cast<cuuint64_t>(p.B)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(p.row_stride) * 4,
+                                   static_cast<cuuint64_t>(p.row_stride) * 4 * p.h_q};
+    const cuuint32_t box[3] = {kTileKeys, kN, 1};
+    if (enc(&kmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float *>(p.scores_in), dims,
+            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
+  } else {
+    {
+      const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(p.cap),
+                                  static_cast<cuuint64_t>(p.h_k), static_cast<cuuint64_t>(p.B)};
+      const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2,
+                                     static_cast<cuuint64_t>(p.k_sh) * 2,
+                                     static_cast<cuuint64_t>(p.k_sb) * 2};
+      const cuuint32_t box[4] = {64, kTileKeys, 1, 1};
+      if (enc(&kmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(p.K), dims, strides,
+              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    }
+    {
+      const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(p.h_q),
+                                  static_cast<cuuint64_t>(p.B)};
+      const cuuint64_t strides[2] = {static_cast<cuuint64_t>(p.q_sh) * 2,
+                                     static_cast<cuuint64_t>(p.q_sb) * 2};
+      const cuuint32_t box[3] = {64, kN, 1};
+      if (enc(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(p.q), dims, strides,
+              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    }
   }
-  {
-    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(p.h_q),
-                                static_cast<cuuint64_t>(p.B)};
-    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(p.q_sh) * 2,
-                                   static_cast<cuuint64_t>(p.q_sb) * 2};
-    const cuuint32_t box[3] = {64, kN, 1};
-    if (enc(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(p.q), dims, strides,
-            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
+#define SAGA_TC_LAUNCH(DD)                                                                    \
+  if (d == DD) {                                                                              \
+    if (mode == kModeDump) return launch_tc<DD, kModeDump, false>(p, kmap, qmap, hm, dev, st); \
+    if (mode == kModeStep)                                                                    \
+      return fs ? launch_tc<DD, kModeStep, true>(p, kmap, qmap, hm, dev, st)                  \
+                : launch_tc<DD, kModeStep, false>(p, kmap, qmap, hm, dev, st);                \
+    return fs ? launch_tc<DD, kModeStepTies, true>(p, kmap, qmap, hm, dev, st)                \
+              : launch_tc<DD, kModeStepTies, false>(p, kmap, qmap, hm, dev, st);              \
   }
-  if (d == 64) {
-    if (mode == kModeDump) return launch_tc<64, kModeDump>(p, kmap, qmap, hm, dev, st);
-    if (mode == kModeStep) return launch_tc<64, kModeStep>(p, kmap, qmap, hm, dev, st);
-    return launch_tc<64, kModeStepTies>(p, kmap, qmap, hm, dev, st);
-  }
-  if (d == 128) {
-    if (mode == kModeDump) return launch_tc<128, kModeDump>(p, kmap, qmap, hm, dev, st);
-    if (mode == kModeStep) return launch_tc<128, kModeStep>(p, kmap, qmap, hm, dev, st);
-    return launch_tc<128, kModeStepTies>(p, kmap, qmap, hm, dev, st);
-  }
+  SAGA_TC_LAUNCH(64)
+  SAGA_TC_LAUNCH(128)
+#undef SAGA_TC_LAUNCH
   return cudaErrorInvalidValue;
 }
 

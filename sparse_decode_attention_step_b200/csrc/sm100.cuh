@@ -42,9 +42,20 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
                : "memory");
 }
 
-// Plain arrive (count 1) with release semantics.
+// Plain arrive (count 1) with release semantics: the arrival becomes
+// visible only after every earlier memory access of this thread has been
+// performed, global loads still in flight included.
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Arrive (count 1) without release semantics: it does not wait for this
+// thread's global loads still in flight. For signals whose data the thread
+// has already consumed (a finished tcgen05.ld, shared-memory values that
+// later instructions of the warp have used).
+__device__ __forceinline__ void mbar_arrive_relaxed(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar))
+               : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
@@ -131,10 +142,15 @@ __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
                : "memory");
 }
 
-// Arrive on `bar` once this thread's earlier cp.async copies have landed
-// (the arrival is counted in advance, so the phase cannot complete before).
-__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
-  asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+// Close this thread's group of cp.async copies issued since the last commit.
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+// Wait until every cp.async group this thread committed has landed (its
+// copies are then visible to this thread).
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
 // Untiled bulk copy global -> shared (no multicast), completing on `bar`.

@@ -102,9 +102,60 @@ def test_stack_layer_full_size(layer):
     lens = synth.seq_lens(w)
     K = dev_cache(w, layer, "K", w.h_k, w.l_kv)
     V = dev_cache(w, layer, "V", w.h_v, w.l_kv)
-    # steps 0..2 plus one more refresh cycle boundary via R=2
+    # three steps at R = 2: refresh, plain step, refresh again
     groups = [(0, 0), (5, 1), (7, 0)]
-    run_chain(w, saga_shape(w), K, V, lens, SynthRows(w, layer), 3, groups, layer=layer)
+    run_chain(w, saga_shape(w), K, V, lens, SynthRows(w, layer), 3, groups, layer=layer, R=2)
+    del K, V
+    torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------------------
+# the calls the benchmark times (no selection mask, no count, scores kept in
+# the workspace) against the checked calls, bit for bit
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("name,layer,groups", [
+    ("llama1b_stack16_b8_128k", 3, [(2, 1), (6, 0)]),
+    ("qwen1p5b_128k", 0, [(0, 0)]),
+    ("llama1b_32k", 0, [(0, 1)])])
+def test_timed_calls_equal_checked_calls_bitwise(name, layer, groups):
+    """One refresh and the plain steps after it, called exactly as the
+    benchmark calls them (sel_mask, sel_count and scores all NULL), must give
+    the same thresholds and outputs, bit for bit, as the same calls with the
+    selection mask, count and score dump the parity checks read; the checked
+    run is then compared with the oracle row by row."""
+    w = synth.WORKLOADS[name]
+    lens = synth.seq_lens(w)
+    K = dev_cache(w, layer, "K", w.h_k, w.l_kv)
+    V = dev_cache(w, layer, "V", w.h_v, w.l_kv)
+    shp = saga_shape(w)
+    steps = 3
+    qs = synth.queries(w, layer, steps)
+    q64 = synth.widen(qs)
+    l = torch.from_numpy(lens).cuda()
+    ws = saga.Workspace(shp, w.N)
+    tau = torch.zeros(w.B, w.h_q, dtype=torch.float32, device="cuda")
+    out = torch.zeros(w.B, w.h_q, w.d, dtype=torch.float32, device="cuda")
+    ch = Chain(shp, K, V, lens, w.N)
+    rows = SynthRows(w, layer)
+    G = w.h_q // w.h_k
+    tau_o = {}
+    for t in range(steps):
+        q = to_dev(qs[t])
+        refresh = t == 0
+        if refresh:
+            saga.refresh_threshold(shp, q, K, l, w.N, tau, ws, V=V, out=out)
+        else:
+            saga.decode_step(shp, q, K, V, l, tau, out, ws)
+        rec = ch.step(q, refresh)
+        assert saga.read_device_error(ws) == 0
+        np.testing.assert_array_equal(tau.cpu().numpy().view(np.uint32), rec.tau.view(np.uint32))
+        np.testing.assert_array_equal(out.cpu().numpy().view(np.uint32), rec.out.view(np.uint32))
+        for (b, kh) in groups:
+            L = int(lens[b])
+            krow = rows.k_row(b, kh, L)
+            for j in range(kh * G, (kh + 1) * G):
+                tau_o[(b, j)] = check_row(rec, q64[t, b, j], krow, rows, b, j, w.h_q, w.h_v, L,
+                                          w.d, w.N, refresh, w.dtype, tau_o.get((b, j)))
     del K, V
     torch.cuda.empty_cache()
 

@@ -11,7 +11,7 @@ import sparse_decode_attention_step_b200 as saga
 import synth
 from synth import device as sdev
 
-from gpu_harness import OUT_TOL, SCORE_TOL, rel_err, to_dev
+from gpu_harness import OUT_TOL, SCORE_TOL, HostRows, SynthRows, rel_err, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -25,7 +25,12 @@ def _built(gpu_lib):
 
 
 def run_topn(w, Kh, Vh, lens, N):
-    B, h_q, d, cap = w.B, w.h_q, w.d, Kh.shape[2]
+    rows = HostRows(synth.widen(Kh), synth.widen(Vh))
+    check_topn(w, to_dev(Kh), to_dev(Vh), Kh.shape[2], lens, N, rows)
+
+
+def check_topn(w, K, V, cap, lens, N, rows, heads=None):
+    B, h_q, d = w.B, w.h_q, w.d
     shp = saga.shape(B, h_q, w.h_k, w.h_v, d, w.dtype, cap)
     ws = saga.Workspace(shp, N)
     qs = synth.queries(w, 0, 1, B=B, h_q=h_q)
@@ -34,25 +39,25 @@ def run_topn(w, Kh, Vh, lens, N):
     cnt = torch.zeros(B, h_q, dtype=torch.int32, device="cuda")
     mask = torch.full((B, h_q, cap), 2, dtype=torch.uint8, device="cuda")
     sc = torch.zeros(B, h_q, cap, dtype=torch.float32, device="cuda")
-    saga.topn_step(shp, to_dev(qs[0]), to_dev(Kh), to_dev(Vh), l, N, out, ws, sel_count=cnt,
+    saga.topn_step(shp, to_dev(qs[0]), K, V, l, N, out, ws, sel_count=cnt,
                    sel_mask=mask, scores=sc)
     torch.cuda.synchronize()
     assert saga.read_device_error(ws) == 0
-    K64, V64, q64 = synth.widen(Kh), synth.widen(Vh), synth.widen(qs[0])
+    q64 = synth.widen(qs[0])
     o, c, m, s = out.cpu().numpy(), cnt.cpu().numpy(), mask.cpu().numpy(), sc.cpu().numpy()
     for b in range(B):
         L = int(lens[b])
-        for j in range(h_q):
+        for j in (range(h_q) if heads is None else heads):
             kh, vh = orc.key_head(j, h_q, w.h_k), orc.value_head(j, h_q, w.h_v)
             assert np.all(m[b, j, L:] == 2)
             kept = np.nonzero(m[b, j, :L] == 1)[0]
             assert c[b, j] == kept.size == min(N, L)
             keys = orc.f32_order_key(s[b, j, :L]).astype(np.float64)   # exact integers
             assert np.array_equal(kept, orc.top_n_exact(keys, N)), (b, j)
-            A = K64[b, kh, :L] @ q64[b, j] / np.sqrt(d)
+            A = rows.k_row(b, kh, L) @ q64[b, j] / np.sqrt(d)
             if L:
                 assert np.max(np.abs(s[b, j, :L] - A)) <= SCORE_TOL * max(1.0, np.max(np.abs(A)))
-            ref = orc.sparse_attend(A[kept], V64[b, vh, kept], np.arange(kept.size))
+            ref = orc.sparse_attend(A[kept], rows.v_rows(b, vh, kept), np.arange(kept.size))
             assert rel_err(o[b, j].astype(np.float64), ref) <= OUT_TOL[w.dtype], (b, j)
 
 
@@ -74,11 +79,15 @@ def test_topn_with_heavy_ties(dtype, d, h_q, h_k, h_v, N):
 
 @pytest.mark.parametrize("name,N", [("llama1b_32k", 1024), ("tiny_f32", 64), ("qwen1p5b_128k", 2048)])
 def test_topn_on_the_workloads(name, N):
+    """At the workloads' full sizes: caches filled on the device by the
+    generator's twin, rows regenerated on the host for the checks."""
     w = synth.WORKLOADS[name]
-    if w.l_kv > 32768:
-        w = synth.Workload(w.name, w.dtype, B=w.B, h_q=w.h_q, h_k=w.h_k, h_v=w.h_v, d=w.d,
-                           l_kv=16384, N=N, R=1, steps=1, seed=w.seed)
     lens = synth.seq_lens(w)
-    Kh = synth.cache(w, 0, "K", w.h_k, w.l_kv, lens)
-    Vh = synth.cache(w, 0, "V", w.h_v, w.l_kv, lens)
-    run_topn(w, Kh, Vh, lens, N)
+    dt = torch.float32 if w.dtype == synth.F32 else torch.int16
+    K = torch.empty(w.B, w.h_k, w.l_kv, w.d, dtype=dt, device="cuda")
+    V = torch.empty(w.B, w.h_v, w.l_kv, w.d, dtype=dt, device="cuda")
+    sdev.fill(K, w, 0, "K")
+    sdev.fill(V, w, 0, "V")
+    check_topn(w, K, V, w.l_kv, lens, N, SynthRows(w, 0))
+    del K, V
+    torch.cuda.empty_cache()

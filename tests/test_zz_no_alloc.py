@@ -1,8 +1,10 @@
 """The allocation-free decode step (saga_decode_step_noalloc), for callers
-that cannot allocate device memory: its output must equal the ordinary
-saga_decode_step's on the same inputs, on two calls in a row (the second call
-finds the first call's leftovers in the shared scratch array). This file is
-named so that pytest collects it last."""
+that cannot allocate device memory: it runs the same plan and kernels as the
+ordinary saga_decode_step, so its output and counts must equal that call's
+bit for bit, on two calls in a row (the second call finds the first call's
+leftovers in the shared scratch array), and pass the oracle's row checks.
+Shapes whose scratch just fits the fixed array run; one sequence more is
+refused. This file is named so that pytest collects it last."""
 import ctypes
 
 import numpy as np
@@ -12,7 +14,27 @@ import torch
 import sparse_decode_attention_step_b200 as saga
 import synth
 
+from gpu_harness import Chain, HostRows, check_row
+
 pytestmark = pytest.mark.gpu
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+
+
+def planned_scratch_bytes(B, h_q, h_k, d, L):
+    """Scratch of a plain step on the tensor-core path: the 256-byte error
+    word and one (m, l, count, pad, acc[d]) float record per (b, j, split),
+    with the persistent plan's split count (148 SMs, up to 128 tiles of 128
+    positions per unit), rounded up to 256 bytes."""
+    rows = B * h_k
+    tiles = rows * -(-L // 128)
+    waves = max(1, -(-tiles // (148 * 128)))
+    s_target = max(1, 148 * waves // rows)
+    split_len = -(-(-(-L // s_target)) // 128) * 128
+    S = -(-L // split_len)
+    return -(-(256 + B * h_q * S * (d + 4) * 4) // 256) * 256
 
 
 def test_noalloc_matches_workspace_step_twice():
@@ -24,33 +46,71 @@ def test_noalloc_matches_workspace_step_twice():
     Kh = synth.cache(w, 0, "K", w.h_k, 3000, lens)
     Vh = synth.cache(w, 0, "V", w.h_v, 3000, lens)
     qs = synth.queries(w, 0, 3)
-    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
-    K, V, l = dev(Kh), dev(Vh), torch.from_numpy(lens).cuda()
+    q64 = synth.widen(qs)
+    rows = HostRows(synth.widen(Kh), synth.widen(Vh))
+    K, V = dev(Kh), dev(Vh)
     shp = saga.shape(w.B, w.h_q, w.h_k, w.h_v, w.d, w.dtype, 3000)
-    ws = saga.Workspace(shp, w.N)
-    tau = torch.zeros(w.B, w.h_q, device="cuda")
-    saga.refresh_threshold(shp, dev(qs[0]), K, l, w.N, tau, ws)
+    ch = Chain(shp, K, V, lens, w.N)             # checked calls: mask, counts, score rows
+    rec0 = ch.step(dev(qs[0]), refresh=True)
+    tau_o = {}
+    for b in range(w.B):
+        for j in range(w.h_q):
+            kh = j // (w.h_q // w.h_k)
+            tau_o[(b, j)] = check_row(rec0, q64[0, b, j], rows.k_row(b, kh, int(lens[b])), rows,
+                                      b, j, w.h_q, w.h_v, int(lens[b]), w.d, w.N, True, w.dtype,
+                                      None)
     for t in (1, 2):                       # two calls in a row
         q = dev(qs[t])
-        ref = torch.zeros(w.B, w.h_q, w.d, device="cuda")
-        ref_cnt = torch.zeros(w.B, w.h_q, dtype=torch.int32, device="cuda")
-        saga.decode_step(shp, q, K, V, l, tau, ref, ws, sel_count=ref_cnt)
+        rec = ch.step(q, refresh=False)    # saga_decode_step on the same tau
         out = torch.full((w.B, w.h_q, w.d), float("nan"), device="cuda")
         cnt = torch.full((w.B, w.h_q), -1, dtype=torch.int32, device="cuda")
-        saga.decode_step_noalloc(shp, q, K, V, l, tau, out, sel_count=cnt)
+        saga.decode_step_noalloc(shp, q, K, V, ch.l, ch.tau, out, sel_count=cnt)
         torch.cuda.synchronize()
-        o, r = out.cpu().numpy(), ref.cpu().numpy()
-        assert np.all(np.isfinite(o))
-        err = np.max(np.abs(o - r), axis=-1) / np.maximum(np.max(np.abs(r), axis=-1), 1e-30)
-        assert np.max(err) <= 2e-3, (t, np.max(err))
-        np.testing.assert_array_equal(cnt.cpu().numpy(), ref_cnt.cpu().numpy())
+        np.testing.assert_array_equal(out.cpu().numpy().view(np.uint32), rec.out.view(np.uint32))
+        np.testing.assert_array_equal(cnt.cpu().numpy(), rec.cnt)
+        for b in range(w.B):
+            for j in range(w.h_q):
+                kh = j // (w.h_q // w.h_k)
+                tau_o[(b, j)] = check_row(rec, q64[t, b, j], rows.k_row(b, kh, int(lens[b])),
+                                          rows, b, j, w.h_q, w.h_v, int(lens[b]), w.d, w.N,
+                                          False, w.dtype, tau_o[(b, j)])
 
 
-def test_noalloc_rejects_shapes_beyond_its_scratch():
-    saga.load()
-    # 64 sequences x 32 heads x 5 splits x 132 floats of split state: 5.4 MB
-    big = saga.shape(64, 32, 2, 8, 128, synth.BF16, 1 << 20)
-    fake = 1 << 40          # never dereferenced: the call is rejected first
-    rc = saga.load().saga_decode_step_noalloc(ctypes.byref(big), fake, fake, fake, fake, fake,
-                                              fake, None, None)
+def test_noalloc_scratch_limit_both_sides():
+    """963 sequences of 128 positions (h_q=16, h_k=2, d=64: one split per
+    sequence) need 4,191,232 bytes of scratch and run; 964 need 4,195,584,
+    more than the 4 MiB array, and are refused before anything runs."""
+    lib = saga.load()
+    limit = saga.NOALLOC_SCRATCH_BYTES
+    L, h_q, h_k, h_v, d = 128, 16, 2, 4, 64
+    under, over = 963, 964
+    assert planned_scratch_bytes(under, h_q, h_k, d, L) <= limit
+    assert planned_scratch_bytes(over, h_q, h_k, d, L) > limit
+
+    big = saga.shape(over, h_q, h_k, h_v, d, synth.BF16, L)
+    fake = 1 << 40          # never dereferenced: the call is refused first
+    rc = lib.saga_decode_step_noalloc(ctypes.byref(big), fake, fake, fake, fake, fake, fake,
+                                      None, None)
     assert rc == saga.SAGA_ERR_WORKSPACE
+
+    w = synth.Workload("noalloc_edge", synth.BF16, B=under, h_q=h_q, h_k=h_k, h_v=h_v, d=d,
+                       l_kv=L, N=16, R=1, steps=2, seed=777)
+    from synth import device as sdev
+    K = torch.empty(under, h_k, L, d, dtype=torch.int16, device="cuda")
+    V = torch.empty(under, h_v, L, d, dtype=torch.int16, device="cuda")
+    sdev.fill(K, w, 0, "K")
+    sdev.fill(V, w, 0, "V")
+    lens = np.full(under, L, dtype=np.int32)
+    lens[::7] = 77                                # ragged tails too
+    shp = saga.shape(under, h_q, h_k, h_v, d, synth.BF16, L)
+    ch = Chain(shp, K, V, lens, w.N, dump=False)
+    qs = synth.queries(w, 0, 2)
+    ch.step(dev(qs[0]), refresh=True)
+    q = dev(qs[1])
+    rec = ch.step(q, refresh=False)
+    out = torch.full((under, h_q, d), float("nan"), device="cuda")
+    cnt = torch.full((under, h_q), -1, dtype=torch.int32, device="cuda")
+    saga.decode_step_noalloc(shp, q, K, V, ch.l, ch.tau, out, sel_count=cnt)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(out.cpu().numpy().view(np.uint32), rec.out.view(np.uint32))
+    np.testing.assert_array_equal(cnt.cpu().numpy(), rec.cnt)
