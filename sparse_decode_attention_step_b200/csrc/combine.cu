@@ -37,8 +37,8 @@ __device__ __forceinline__ void load_slice(const float *p, float (&v)[VPL]) {
 template <int D>
 __global__ void __launch_bounds__(kThreads)
 combine_kernel(const float *__restrict__ partials, const int32_t *__restrict__ l_kv,
-               float *__restrict__ out, int32_t *__restrict__ sel_count, int h_q, int S,
-               int64_t split_len, int64_t cap, int64_t max_l_kv) {
+               float *__restrict__ out, int32_t *__restrict__ sel_count, int32_t *abort_word,
+               int h_q, int S, int64_t split_len, int64_t cap, int64_t max_l_kv) {
   constexpr int VPL = D / 32;                  // output elements per lane
   constexpr int R = D + kRecPad;
   __shared__ float red[kWarps];
@@ -120,22 +120,24 @@ combine_kernel(const float *__restrict__ partials, const int32_t *__restrict__ l
     out[static_cast<int64_t>(bj) * D + tid] = o;
     if (tid == 0 && sel_count != nullptr) sel_count[bj] = nt;
   }
+  // the step is over (its gather read the abort word before this launch
+  // began): clear the word for the next step
+  if (abort_word != nullptr && bj == 0 && tid == 0) *abort_word = 0;
 }
 
 }  // namespace
 
-cudaError_t launch_combine(const float *partials, const int32_t *l_kv, int32_t *err,
+cudaError_t launch_combine(const float *partials, const int32_t *l_kv, int32_t *abort_word,
                            float *out, int32_t *sel_count, int B, int h_q, int d, int S,
                            int64_t split_len, int64_t cap, int64_t max_l_kv,
                            cudaStream_t st) {
-  (void)err;
   const dim3 grid(B * h_q), block(kThreads);
   if (d == 64)
-    return launch_pdl(combine_kernel<64>, grid, block, 0, st, partials, l_kv, out, sel_count, h_q,
-                      S, split_len, cap, max_l_kv);
+    return launch_pdl(combine_kernel<64>, grid, block, 0, st, partials, l_kv, out, sel_count,
+                      abort_word, h_q, S, split_len, cap, max_l_kv);
   if (d == 128)
-    return launch_pdl(combine_kernel<128>, grid, block, 0, st, partials, l_kv, out, sel_count, h_q,
-                      S, split_len, cap, max_l_kv);
+    return launch_pdl(combine_kernel<128>, grid, block, 0, st, partials, l_kv, out, sel_count,
+                      abort_word, h_q, S, split_len, cap, max_l_kv);
   return cudaErrorInvalidValue;
 }
 

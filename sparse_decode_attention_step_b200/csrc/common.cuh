@@ -25,7 +25,12 @@ struct StepParams {
   uint8_t *sel_mask;        // nullable [B][h_q][row_stride]
   uint32_t *hist;           // nullable [B][h_q][256]: dump mode adds the top-byte histogram
                             // of each score row's order keys
+  uint32_t *lmask;          // step modes (tensor-core scan): [B * h_q][nblk] kept-position
+                            // mask of every 32-position block of each query head's row
+  float *lscore;            // [B * h_q][nblk * 32] kept scores, at each key's rank in its block
+  int64_t nblk;             // 32-position blocks per row (lists)
   int32_t *err;             // device error word
+  int32_t *abort;           // the step's abort word: set when a bounded wait gives up
   int64_t q_sb, q_sh, k_sb, k_sh, v_sb, v_sh;
   int64_t cap, max_l_kv, row_stride;
   int64_t split_len;
@@ -35,6 +40,22 @@ struct StepParams {
 
 // Clamp a device-side sequence length into [0, min(cap, max_l_kv)] and
 // record any violation in the error word.
+// Gather kernel parameters: the kept lists of a tensor-core scan, the V
+// cache and the per-split records to write (strides in elements).
+struct GatherParams {
+  const uint16_t *V;
+  int64_t v_sb, v_sh;
+  const int32_t *l_kv;
+  int64_t cap, max_l_kv;
+  const uint32_t *lmask;    // [B * h_q][nblk]
+  const float *lscore;      // [B * h_q][nblk * 32]
+  int64_t nblk;
+  float *partials;          // [B][h_q][SB][d + kRecPad]
+  const int32_t *abort;     // the scan's abort word
+  int32_t B, h_q, h_v, SB;
+  int64_t blk_per_split;    // 32-position blocks per split
+};
+
 __device__ __forceinline__ int64_t clamp_len(const StepParams &p, int b) {
   int64_t L = p.l_kv[b];
   int64_t hi = p.cap < p.max_l_kv ? p.cap : p.max_l_kv;

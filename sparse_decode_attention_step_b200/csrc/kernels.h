@@ -23,17 +23,22 @@ cudaError_t launch_saga_split(const StepParams &p, int mode, int dtype, int d, i
 // when p.scores_in is set. Shapes it takes: saga_tc_supports.
 cudaError_t launch_saga_tc(const StepParams &p, int mode, int d, cudaStream_t st);
 
-// bf16 caches, d in {64, 128}, G = h_q / h_k <= 16, and the query heads of a
-// group fit four lane groups: (h_v / h_k) * ceil((h_q / h_v) / 4) <= 4.
+// bf16 caches, d in {64, 128}, G = h_q / h_k <= 16 (one MMA's N), h_q a
+// multiple of h_v and h_v of h_k.
 bool saga_tc_supports(int dtype, int d, int h_q, int h_k, int h_v);
+
+// The V-row half of a tensor-core step: per-split records from the scan's
+// kept lists (gather.cu).
+cudaError_t launch_gather(const GatherParams &p, int d, cudaStream_t st);
 
 // The tensor-core step kernel can stream stored score rows (StepParams::
 // scores_in, [B][h_q][row_stride] fp32) in place of K: 16-byte aligned rows
 // whose stride is a multiple of four floats.
 bool saga_tc_scores_streamable(const float *rows, int64_t row_stride);
 
-// Merge the per-split states of every (b, j) into out and sel_count.
-cudaError_t launch_combine(const float *partials, const int32_t *l_kv, int32_t *err,
+// Merge the per-split states of every (b, j) into out and sel_count; when
+// abort_word is given, clear it afterwards (the step that set it is over).
+cudaError_t launch_combine(const float *partials, const int32_t *l_kv, int32_t *abort_word,
                            float *out, int32_t *sel_count, int B, int h_q, int d, int S,
                            int64_t split_len, int64_t cap, int64_t max_l_kv,
                            cudaStream_t st);

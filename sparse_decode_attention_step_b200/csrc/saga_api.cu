@@ -24,9 +24,17 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 struct Plan {
-  int S;                    // splits per (b, key head)
-  int64_t split_len;        // positions per split
-  size_t off_partials, off_scores, off_hist, off_tau, off_tie, total;
+  int S;                    // scan / split-kernel units per (b, key head)
+  int64_t split_len;        // positions per unit
+  // tensor-core path: the gather kernel's own splits of a row
+  bool lists;               // the scan writes per-head kept lists
+  int SB;                   // gather splits per (b, query head)
+  int64_t blk_per_split;    // 32-position blocks per gather split
+  int64_t nblk;             // 32-position blocks per row
+  // the records the combine merges: comb_S per (b, j), comb_split_len positions each
+  int comb_S;
+  int64_t comb_split_len;
+  size_t off_partials, off_lmask, off_lscore, off_scores, off_hist, off_tau, off_tie, total;
 };
 
 bool use_tc(const saga_shape &s);
@@ -38,9 +46,14 @@ bool use_tc(const saga_shape &s);
 // (`ctas_per_sm`, at most kGridCtasPerSm, which sizes the workspace): those
 // kernels hide their load latency only with every resident slot filled, and
 // more splits than slots only add waves and combine work.
-// Persistent tensor-core kernel: at most one unit per SM and wave, units of up
-// to about kPersistTiles tiles, since every unit ends with a merge of the
-// workers' states.
+// Persistent tensor-core scan: at most one unit per SM and wave, units of up
+// to about kPersistTiles tiles. Its gather kernel splits each (b, query head)
+// row on its own, into at most kGatherCtas CTAs in all (one wave, six
+// resident per SM) where the rows allow, each at least kGatherMinBlocks
+// blocks of 32 positions long; the combine merges the gather's records.
+constexpr int64_t kGatherCtas = 6 * kSms;
+constexpr int64_t kGatherMinBlocks = 8;
+
 Plan make_plan(const saga_shape &s, bool persistent, int64_t ctas_per_sm = kGridCtasPerSm) {
   Plan p{};
   const int64_t rows = static_cast<int64_t>(s.B) * s.h_k;
@@ -57,9 +70,25 @@ Plan make_plan(const saga_shape &s, bool persistent, int64_t ctas_per_sm = kGrid
   }
   p.split_len = ceil_div(ceil_div(L, s_target), kTileKeys) * kTileKeys;
   p.S = static_cast<int>(ceil_div(L, p.split_len));
+  p.comb_S = p.S;
+  p.comb_split_len = p.split_len;
+  p.nblk = ceil_div(L, 32);
+  if (persistent && saga_tc_supports(s.dtype, s.d, s.h_q, s.h_k, s.h_v)) {
+    p.lists = true;
+    const int64_t items = static_cast<int64_t>(s.B) * s.h_q;
+    const int64_t max_sb = std::max<int64_t>(1, p.nblk / kGatherMinBlocks);
+    const int64_t sb = std::min(max_sb, std::max<int64_t>(1, kGatherCtas / items));
+    p.blk_per_split = ceil_div(p.nblk, sb);
+    p.SB = static_cast<int>(ceil_div(p.nblk, p.blk_per_split));
+    p.comb_S = p.SB;
+    p.comb_split_len = p.blk_per_split * 32;
+  }
   const size_t rec = static_cast<size_t>(s.d + kRecPad) * sizeof(float);
-  p.off_partials = kAlign;   // [0, 256): device error word
-  p.off_scores = align_up(p.off_partials + static_cast<size_t>(s.B) * s.h_q * p.S * rec);
+  const size_t lists = p.lists ? static_cast<size_t>(s.B) * s.h_q * p.nblk : 0;
+  p.off_partials = kAlign;   // [0, 256): device error word, then the step's abort word
+  p.off_lmask = align_up(p.off_partials + static_cast<size_t>(s.B) * s.h_q * p.comb_S * rec);
+  p.off_lscore = align_up(p.off_lmask + lists * sizeof(uint32_t));
+  p.off_scores = align_up(p.off_lscore + lists * 32 * sizeof(float));
   p.off_hist = align_up(p.off_scores + static_cast<size_t>(s.B) * s.h_q * s.max_l_kv * sizeof(float));
   p.off_tau = align_up(p.off_hist + static_cast<size_t>(s.B) * s.h_q * 256 * sizeof(uint32_t));
   p.off_tie = align_up(p.off_tau + static_cast<size_t>(s.B) * s.h_q * sizeof(float));
@@ -70,9 +99,10 @@ Plan make_plan(const saga_shape &s, bool persistent, int64_t ctas_per_sm = kGrid
 // The plan of the SAGA calls (step, refresh, debug scores) of a shape.
 Plan saga_plan(const saga_shape &s) { return make_plan(s, use_tc(s)); }
 
-// One workspace serves every call of a shape: the larger of the two plans.
+// One workspace serves every call of a shape: the larger of the step's plan
+// and the grid-per-split plan (dense calls, at most kGridCtasPerSm units per SM).
 size_t workspace_bytes(const saga_shape &s) {
-  return std::max(make_plan(s, true).total, make_plan(s, false).total);
+  return std::max(saga_plan(s).total, make_plan(s, false).total);
 }
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -114,9 +144,16 @@ saga_status check_inputs(const saga_shape &s, const void *q, const void *K, cons
 StepParams base_params(const saga_shape &s, const Plan &pl, const void *q, const void *K,
                        const void *V, const int32_t *l_kv, void *ws) {
   StepParams p{};
+  char *wsb = static_cast<char *>(ws);
   p.q = q; p.K = K; p.V = V; p.l_kv = l_kv;
   p.err = static_cast<int32_t *>(ws);
-  p.partials = reinterpret_cast<float *>(static_cast<char *>(ws) + pl.off_partials);
+  p.abort = static_cast<int32_t *>(ws) + 1;
+  p.partials = reinterpret_cast<float *>(wsb + pl.off_partials);
+  if (pl.lists) {
+    p.lmask = reinterpret_cast<uint32_t *>(wsb + pl.off_lmask);
+    p.lscore = reinterpret_cast<float *>(wsb + pl.off_lscore);
+    p.nblk = pl.nblk;
+  }
   p.q_sb = s.q_stride_b; p.q_sh = s.q_stride_h;
   p.k_sb = s.k_stride_b; p.k_sh = s.k_stride_h;
   p.v_sb = s.v_stride_b; p.v_sh = s.v_stride_h;
@@ -144,13 +181,28 @@ cudaError_t launch_split(const saga_shape &s, const StepParams &p, int mode, cud
   return launch_saga_split(p, mode, s.dtype, s.d, group_pad(s), st);
 }
 
-// Select + PV over the stored thresholds, then the combine.
+// Select + PV over the stored thresholds, then the combine. Tensor-core
+// shapes: the scan kernel writes the kept lists, the gather kernel the
+// records; other shapes: the SIMT split kernel does both.
 saga_status run_step(const saga_shape &s, const Plan &pl, StepParams p, int mode,
                      float *out, int32_t *sel_count, cudaStream_t st) {
+  const bool tc = mode != kModeFromScores && use_tc(s);
   cudaError_t e = launch_split(s, p, mode, st);
-  if (e != cudaSuccess) return cuda_fail(e, p.scores_in ? "step kernel (stored scores)" : "step kernel");
-  return cuda_check(launch_combine(p.partials, p.l_kv, p.err, out, sel_count, s.B, s.h_q, s.d,
-                                   pl.S, pl.split_len, s.cap, s.max_l_kv, st),
+  if (e != cudaSuccess)
+    return cuda_fail(e, !tc ? "split kernel" : (p.scores_in ? "scan kernel (stored scores)" : "scan kernel"));
+  if (tc) {
+    GatherParams g{};
+    g.V = static_cast<const uint16_t *>(p.V);
+    g.v_sb = p.v_sb; g.v_sh = p.v_sh;
+    g.l_kv = p.l_kv; g.cap = p.cap; g.max_l_kv = p.max_l_kv;
+    g.lmask = p.lmask; g.lscore = p.lscore; g.nblk = p.nblk;
+    g.partials = p.partials; g.abort = p.abort;
+    g.B = s.B; g.h_q = s.h_q; g.h_v = s.h_v; g.SB = pl.SB;
+    g.blk_per_split = pl.blk_per_split;
+    if ((e = launch_gather(g, s.d, st)) != cudaSuccess) return cuda_fail(e, "gather kernel");
+  }
+  return cuda_check(launch_combine(p.partials, p.l_kv, tc ? p.abort : nullptr, out, sel_count, s.B,
+                                   s.h_q, s.d, pl.comb_S, pl.comb_split_len, s.cap, s.max_l_kv, st),
                     "combine kernel");
 }
 
@@ -169,7 +221,7 @@ saga_status run_dense(const saga_shape &s, const void *q, const void *K, const v
   StepParams p = base_params(s, pl, q, K, V, l_kv, ws);
   cudaError_t e = launch_dense_split(p, s.dtype, s.d, st);
   if (e != cudaSuccess) return cuda_fail(e, "dense kernel");
-  return cuda_check(launch_combine(p.partials, l_kv, p.err, out, nullptr, s.B, s.h_q, s.d, pl.S,
+  return cuda_check(launch_combine(p.partials, l_kv, nullptr, out, nullptr, s.B, s.h_q, s.d, pl.S,
                                    pl.split_len, s.cap, s.max_l_kv, st),
                     "combine kernel");
 }

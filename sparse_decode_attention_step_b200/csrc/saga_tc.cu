@@ -1,6 +1,7 @@
-// Tensor-core split kernel for bf16 caches (sm_100a): Eq. 2 scores,
-// Atop-N item 1 compare, Eq. 7 sparse softmax with the V gather, and the
-// per-split online-softmax states, with the score contraction on tcgen05.
+// Tensor-core scan kernel for bf16 caches (sm_100a): the K-streaming half of
+// the decode step. Eq. 2 scores on tcgen05, the Atop-N item 1 compare, and
+// the kept lists that the gather kernel (gather.cu) turns into Eq. 7
+// per-split states; for a refresh, the score rows and their histograms.
 //
 // Persistent: one CTA per SM walks the work units (sequence b, key head kh,
 // split s of l_kv) u = blockIdx.x, blockIdx.x + gridDim.x, ... Warp roles:
@@ -16,17 +17,15 @@
 //   workers     4 x kRanks warps. Tile g belongs to rank g % kRanks; each of
 //               the four warps of that rank reads its TMEM lane quarter
 //               (32 keys x 16 heads), scales by 1/sqrt(d), compares with tau
-//               and gathers V for its own kept keys: lane group v (8 lanes)
-//               owns up to four query heads that share one value head, so
-//               each kept V row is read once for all of them, and keeps their
-//               online-softmax states (m, l, count, acc) in registers.
+//               and, for each query head, writes the 32-bit mask of kept
+//               keys of its 32-position block and each kept score at the
+//               key's rank within the block.
 //
-// Each worker folds a quarter tile's kept rows in rounds of kRows V rows per
-// lane group (empty rows and heads no lane group kept are skipped, and the
-// states are rescaled only when a round raises a maximum). At the end of a
-// unit every worker writes its states to shared memory, the per-head
-// weights e^{m_w - m} are formed once, and all workers write the unit's
-// (m, l, count, acc) records.
+// The scan never waits for a V row: the V gather runs in its own kernel at
+// full occupancy, where enough rows can be in flight to cover the latency
+// of random row reads under load (about 2-3 us), which a warp that also
+// scans cannot do. The lists are written at fixed places, so the step is
+// deterministic.
 //
 // Modes: dump (score rows and per-row top-byte histograms of the order keys,
 // for a refresh), step (keep A >= tau), step with ties (exact top-N: keep A
@@ -37,10 +36,10 @@
 //
 // Query heads beyond the group (G < 16) are rows of other heads or zero rows
 // of Q; their tau is +inf, so they are never kept, and they are never dumped.
-// Every wait is bounded; on a timeout the CTA sets SAGA_DEVERR_TIMEOUT, all
-// roles stop after the copies and MMAs in flight have landed, and the
-// workers write poisoned records (m = +inf, count = -1) for every unit the
-// CTA had left, which the combine turns into NaN outputs and counts of -1.
+// Every wait is bounded; on a timeout the CTA sets SAGA_DEVERR_TIMEOUT and the
+// step's abort word, and all roles stop after the copies and MMAs in flight
+// have landed; the gather then writes poisoned records (m = +inf, count = -1),
+// which the combine turns into NaN outputs and counts of -1.
 #include <cuda.h>
 
 #include <atomic>
@@ -58,9 +57,6 @@ constexpr int kTileKeys = 128;
 constexpr int kN = 16;                      // MMA N: query heads of a group, padded
 constexpr int kWorkerBar = 1;               // named barrier of the worker warps
 constexpr uint32_t kIdesc = sm100::idesc_bf16_f32(kTileKeys, kN);
-constexpr float kLog2e = 1.4426950408889634f;
-
-constexpr int cmax(int a, int b) { return a > b ? a : b; }
 
 template <int D>
 struct Cfg {
@@ -76,17 +72,10 @@ struct Cfg {
   static constexpr int kTileBytes = kBoxes * kBoxBytes;
   static constexpr int kQBoxBytes = kN * 128;
   static constexpr int kQBytes = kBoxes * kQBoxBytes;
-  static constexpr int kRows = 4;                              // kept V rows in flight per lane group
   static constexpr int kScoreTileBytes = kN * kTileKeys * 4;   // FS stage: [16][128] fp32
   static_assert(kScoreTileBytes <= kTileBytes, "a score tile fits a stage");
-  static constexpr int CPL = D / 64;                           // 16-byte chunks per lane per V row
-  static constexpr int EPL = 8 * CPL;                          // V row elements per lane
-  static constexpr int kRec = D + kRecPad;
-  static constexpr int kStateFloats = kN * kRec;               // one warp's 16 head states
-  static constexpr int kScoreBytes = kWorkers * 2 * 32 * kN * 4;   // two kept-score row sets per warp
-  static constexpr int kMergeBytes = kWorkers * (kStateFloats + kN) * 4;  // states + weights
-  static constexpr int kHistBytes = kN * 256 * 4;
-  static constexpr int kScratchBytes = cmax(cmax(kScoreBytes, kMergeBytes), kHistBytes);
+  static constexpr int kHistBytes = kN * 256 * 4;              // dump mode: per-head top-byte bins
+  static constexpr int kScratchBytes = kHistBytes;
 };
 
 template <int D>
@@ -112,19 +101,6 @@ struct Layout {
   static_assert(alloc <= 227 * 1024, "shared memory of one CTA");
   static_assert(off_hdr % 16 == 0 && off_q % 1024 == 0, "operand alignment");
 };
-
-// Lane group v of a worker warp owns query heads hbase[v] .. hbase[v] + nh[v] - 1
-// of the group, all reading value head kh * (h_v / h_k) + vs[v]; smask[v] is
-// the same set as a 16-bit mask.
-struct HeadMap {
-  int hbase[4], nh[4], vs[4];
-  uint32_t smask[4];
-};
-
-// a[v] for a lane-dependent v without indexing the parameter array
-__device__ __forceinline__ int pick4(const int (&a)[4], int v) {
-  return v == 0 ? a[0] : (v == 1 ? a[1] : (v == 2 ? a[2] : a[3]));
-}
 
 struct Unit {
   int b, kh, s;
@@ -160,7 +136,10 @@ __device__ __forceinline__ bool aborted(Header<D> *h) {
 
 template <int D>
 __device__ __forceinline__ void fail(const StepParams &p, Header<D> *h) {
-  if (!aborted(h)) atomicOr(p.err, SAGA_DEVERR_TIMEOUT);
+  if (!aborted(h)) {
+    atomicOr(p.err, SAGA_DEVERR_TIMEOUT);
+    if (p.abort != nullptr) atomicExch(p.abort, 1);   // the gather poisons this step's records
+  }
   *reinterpret_cast<volatile int *>(&h->abort) = 1;
 }
 
@@ -204,46 +183,12 @@ __device__ __forceinline__ void workers_sync() {
   sm100::named_bar(kWorkerBar, Cfg<D>::kWorkers * 32);
 }
 
-// Kept-score row of key k in a worker's scratch: 16 floats, 16-byte quads
-// rotated by the key so the four row stores of a warp spread over the banks.
-__device__ __forceinline__ int score_slot(int k, int h) {
-  return k * kN + ((((h >> 2) ^ (k >> 1)) & 3) << 2) + (h & 3);
-}
-
-// One worker state (m, l, count, acc over its lane's slice) into a record
-// laid out as {m, l, count, pad, acc[D]}; lane c8 == 0 writes the scalars.
-template <int EPL>
-__device__ __forceinline__ void put_state(float *r, int c8, float m, float l, int cnt,
-                                          const float (&acc)[EPL]) {
-  if (c8 == 0) {
-    r[0] = m;
-    r[1] = l;
-    r[2] = __int_as_float(cnt);
-    r[3] = 0.f;
-  }
-#pragma unroll
-  for (int cc = 0; cc < EPL / 8; ++cc) {
-    float4 *dst = reinterpret_cast<float4 *>(r + kRecPad + (c8 + 8 * cc) * 8);
-    dst[0] = make_float4(acc[8 * cc], acc[8 * cc + 1], acc[8 * cc + 2], acc[8 * cc + 3]);
-    dst[1] = make_float4(acc[8 * cc + 4], acc[8 * cc + 5], acc[8 * cc + 6], acc[8 * cc + 7]);
-  }
-}
-
-// Poisoned record: the combine turns it into a NaN output and a count of -1.
-__device__ __forceinline__ void put_poison(float *r) {
-  r[0] = INFINITY;
-  r[1] = __int_as_float(0x7fc00000);
-  r[2] = __int_as_float(-1);
-  r[3] = 0.f;
-}
-
 template <int D, int MODE, bool FS>
 __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
 saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
-               const __grid_constant__ CUtensorMap qmap, const HeadMap hm) {
+               const __grid_constant__ CUtensorMap qmap) {
   using C = Cfg<D>;
   using Lo = Layout<D>;
-  constexpr int CPL = C::CPL, EPL = C::EPL, kRows = C::kRows;
   constexpr bool kDump = MODE == kModeDump;
   static_assert(!(kDump && FS), "the dump reads K");
 
@@ -257,7 +202,6 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = p.h_q / p.h_k;
-  const int vpg = p.h_v / p.h_k;
   const int n_units = p.B * p.h_k * p.S;
 
   // ---- set-up (touches no global memory) ---------------------------------
@@ -396,105 +340,11 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
     const int widx = warp - 2;
     const int quarter = warp & 3;             // TMEM lanes (keys) this warp reads
     const int rank = widx >> 2;
-    const int v = lane >> 3, c8 = lane & 7;
-    const int hbase = pick4(hm.hbase, v), nh = pick4(hm.nh, v), vsl = pick4(hm.vs, v);
-    const bool quad = (hbase & 3) == 0 && nh == 4;   // the heads are one 16-byte quad of a row
-    // two kept-score row sets, used in turn: the rows in flight keep theirs
-    float *rows_base = scratch + widx * 2 * 32 * kN;
+    const uint32_t lt_mask = (1u << lane) - 1u;
     uint32_t g = 0;
     bool bad = false;
 
-    float m[4], l[4], acc[4][EPL];
-    int cnt[4];
-    const uint16_t *vrow = nullptr;
-    // Fold the kept keys `mine` of this lane group (keys t0 + bit) into the
-    // lane group's online-softmax states, kRows V rows in flight per round.
-    auto gather = [&](uint32_t mine, int64_t t0, int64_t t_any, const float *rows) {
-      const int nmax = static_cast<int>(__reduce_max_sync(0xffffffffu, __popc(mine)));
-      for (int r0 = 0; r0 < nmax; r0 += kRows) {
-        uint4 raw[kRows][CPL];
-        float sc[kRows][4];
-#pragma unroll
-        for (int r = 0; r < kRows; ++r) {
-          if (r0 + r >= nmax) {
-#pragma unroll
-            for (int a = 0; a < 4; ++a) sc[r][a] = -INFINITY;
-            continue;
-          }
-          const int kk = mine != 0u ? __ffs(mine) - 1 : -1;
-
-          mine &= mine - 1u;
-          // idle slots re-read a row of the unit, which always exists
-          const int64_t tr = kk >= 0 ? t0 + kk : t_any;
-#pragma unroll
-          for (int cc = 0; cc < CPL; ++cc)
-            raw[r][cc] = __ldg(reinterpret_cast<const uint4 *>(vrow + tr * D) + c8 + 8 * cc);
-          const int ks = kk >= 0 ? kk : 0;
-          if (quad) {
-            const float4 q4 = *reinterpret_cast<const float4 *>(rows + score_slot(ks, hbase));
-            sc[r][0] = kk >= 0 ? q4.x : -INFINITY;
-            sc[r][1] = kk >= 0 ? q4.y : -INFINITY;
-            sc[r][2] = kk >= 0 ? q4.z : -INFINITY;
-            sc[r][3] = kk >= 0 ? q4.w : -INFINITY;
-          } else {
-#pragma unroll
-            for (int a = 0; a < 4; ++a) {
-              const int hd = min(hbase + a, kN - 1);
-              sc[r][a] = (kk >= 0 && a < nh) ? rows[score_slot(ks, hd)] : -INFINITY;
-            }
-          }
-        }
-        float mnew[4];
-        bool grow = false;
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          float mx = sc[0][a];
-#pragma unroll
-          for (int r = 1; r < kRows; ++r) mx = fmaxf(mx, sc[r][a]);
-          mnew[a] = fmaxf(m[a], mx);
-          grow |= mnew[a] != m[a];
-        }
-        if (__any_sync(0xffffffffu, grow)) {
-#pragma unroll
-          for (int a = 0; a < 4; ++a) {
-            const float corr = mnew[a] == m[a] ? 1.f : exp2f((m[a] - mnew[a]) * kLog2e);
-            m[a] = mnew[a];
-            l[a] *= corr;
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) acc[a][e] *= corr;
-          }
-        }
-
-#pragma unroll
-        for (int r = 0; r < kRows; ++r) {
-          if (r0 + r >= nmax) break;
-          float vf[EPL];
-
-#pragma unroll
-          for (int cc = 0; cc < CPL; ++cc) {
-            const uint4 x = raw[r][cc];
-            vf[8 * cc + 0] = bf16lo(x.x); vf[8 * cc + 1] = bf16hi(x.x);
-            vf[8 * cc + 2] = bf16lo(x.y); vf[8 * cc + 3] = bf16hi(x.y);
-            vf[8 * cc + 4] = bf16lo(x.z); vf[8 * cc + 5] = bf16hi(x.z);
-            vf[8 * cc + 6] = bf16lo(x.w); vf[8 * cc + 7] = bf16hi(x.w);
-          }
-#pragma unroll
-          for (int a = 0; a < 4; ++a) {
-            const bool in = sc[r][a] != -INFINITY;
-            if (!__any_sync(0xffffffffu, in)) continue;
-            const float pw = in ? exp2f((sc[r][a] - m[a]) * kLog2e) : 0.f;
-
-            l[a] += pw;
-            cnt[a] += in ? 1 : 0;
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) acc[a][e] = fmaf(pw, vf[e], acc[a][e]);
-          }
-        }
-      }
-    };
-
-    int u = blockIdx.x;
-    for (; u < n_units; u += gridDim.x) {
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
       Unit un;
       if (!unit_at(p, u, false, un)) continue;
       const int j0 = un.kh * G;
@@ -506,15 +356,6 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
         }
         workers_sync<D>();
       }
-#pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        m[a] = -INFINITY; l[a] = 0.f; cnt[a] = 0;
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) acc[a][e] = 0.f;
-      }
-      vrow = static_cast<const uint16_t *>(p.V) + un.b * p.v_sb +
-             static_cast<int64_t>(un.kh * vpg + vsl) * p.v_sh;
-      int n_mine = 0;
 
       const int first = (rank - static_cast<int>(g % C::kRanks) + C::kRanks) % C::kRanks;
       for (int i = first; i < un.n_tiles; i += C::kRanks) {
@@ -572,8 +413,6 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
         }
 
         // ---- compare: the heads that keep this lane's key --------------------
-        float *rows = rows_base + (n_mine & 1) * 32 * kN;
-        ++n_mine;
         uint32_t sel = 0;
         {
           const float4 *tq = reinterpret_cast<const float4 *>(h->tau);
@@ -599,99 +438,44 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
             }
           }
         }
-        if (sel != 0u) {
-#pragma unroll
-          for (int a4 = 0; a4 < kN / 4; ++a4)
-            *reinterpret_cast<float4 *>(rows + score_slot(lane, 4 * a4)) =
-                make_float4(A[4 * a4], A[4 * a4 + 1], A[4 * a4 + 2], A[4 * a4 + 3]);
-        }
         if (p.sel_mask != nullptr && valid) {
           for (int a = 0; a < G; ++a)
             p.sel_mask[row0 + a * p.row_stride + t] = static_cast<uint8_t>((sel >> a) & 1u);
         }
-        uint32_t mine = 0;
+        // ---- the kept lists of this 32-position block, per query head: the
+        // mask, and each kept score at the key's rank within the block
+        // (quarters of the last tile that lie past the row's nblk blocks
+        // belong to no block of the row: nothing is written for them)
+        const int64_t blk = t0 >> 5;
+        if (blk < p.nblk) {
+          const int64_t hrow0 = static_cast<int64_t>(un.b * p.h_q + j0) * p.nblk + blk;
+          uint32_t mymask = 0;
 #pragma unroll
-        for (int vv = 0; vv < 4; ++vv) {
-          const uint32_t bl = __ballot_sync(0xffffffffu, (sel & hm.smask[vv]) != 0u);
-          if (v == vv) mine = bl;
+          for (int a = 0; a < kN; ++a) {
+            if (a >= G) break;
+            const uint32_t bl = __ballot_sync(0xffffffffu, (sel >> a) & 1u);
+            if (lane == a) mymask = bl;
+            if ((bl >> lane) & 1u) p.lscore[(hrow0 + a * p.nblk) * 32 + __popc(bl & lt_mask)] = A[a];
+          }
+          if (lane < G) p.lmask[hrow0 + lane * p.nblk] = mymask;
         }
         // FS: every lane's scores have gone into `sel` and the ballots above,
         // so the stage can be refilled
         if (FS && lane == 0) sm100::mbar_arrive(&h->empty[gg % C::kStages]);
-        __syncwarp();
-        gather(mine, t0, un.t_begin, rows);
-        __syncwarp();            // rows read before a later tile overwrites them
       }
       g += un.n_tiles;
 
       // ---- end of unit -------------------------------------------------------
-      if (workers_any<D>(bad || aborted(h))) { bad = true; break; }
-      if (kDump) {
-        if (p.hist != nullptr) {
-          uint32_t *hs = reinterpret_cast<uint32_t *>(scratch);
-          for (int i = widx * 32 + lane; i < kN * 256; i += C::kWorkers * 32) {
-            const uint32_t c = hs[i];
-            if (c != 0u && i / 256 < G)
-              atomicAdd(&p.hist[static_cast<int64_t>(un.b * p.h_q + j0 + i / 256) * 256 + (i % 256)], c);
-            hs[i] = 0u;
-          }
-          workers_sync<D>();
+      if (workers_any<D>(bad || aborted(h))) break;
+      if (kDump && p.hist != nullptr) {
+        uint32_t *hs = reinterpret_cast<uint32_t *>(scratch);
+        for (int i = widx * 32 + lane; i < kN * 256; i += C::kWorkers * 32) {
+          const uint32_t c = hs[i];
+          if (c != 0u && i / 256 < G)
+            atomicAdd(&p.hist[static_cast<int64_t>(un.b * p.h_q + j0 + i / 256) * 256 + (i % 256)], c);
+          hs[i] = 0u;
         }
-        continue;
-      }
-      // merge: every worker's 16 head states into shared memory, then
-      // per head the weights e^{m_w - m} of the workers, then the records
-      {
-        float *st = scratch + widx * C::kStateFloats;
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-          put_state<EPL>(st + (v * 4 + a) * C::kRec, c8, m[a], l[a], cnt[a], acc[a]);
-      }
-      workers_sync<D>();
-      float *wts = scratch + C::kWorkers * C::kStateFloats;       // [kN][kWorkers]
-      const int tw = widx * 32 + lane;
-      if (tw < kN) {
-        const int slot = tw, sv = slot >> 2, sa = slot & 3;
-        float mm = -INFINITY;
-        for (int w = 0; w < C::kWorkers; ++w) mm = fmaxf(mm, scratch[w * C::kStateFloats + slot * C::kRec]);
-        float ll = 0.f;
-        int nn = 0;
-        for (int w = 0; w < C::kWorkers; ++w) {
-          const float *r = scratch + w * C::kStateFloats + slot * C::kRec;
-          const float wt = r[0] == -INFINITY ? 0.f : exp2f((r[0] - mm) * kLog2e);
-          wts[slot * C::kWorkers + w] = wt;
-          ll = fmaf(wt, r[1], ll);
-          nn += __float_as_int(r[2]);
-        }
-        if (sa < pick4(hm.nh, sv)) {
-          const int j = j0 + pick4(hm.hbase, sv) + sa;
-          float *rec = p.partials + (static_cast<int64_t>(un.b * p.h_q + j) * p.S + un.s) * C::kRec;
-          rec[0] = mm;
-          rec[1] = ll;
-          rec[2] = __int_as_float(nn);
-          rec[3] = 0.f;
-        }
-      }
-      workers_sync<D>();
-      for (int idx = tw; idx < kN * D; idx += C::kWorkers * 32) {
-        const int slot = idx / D, dd = idx % D, sv = slot >> 2, sa = slot & 3;
-        if (sa >= pick4(hm.nh, sv)) continue;
-        float a = 0.f;
-        for (int w = 0; w < C::kWorkers; ++w)
-          a = fmaf(wts[slot * C::kWorkers + w],
-                   scratch[w * C::kStateFloats + slot * C::kRec + kRecPad + dd], a);
-        const int j = j0 + pick4(hm.hbase, sv) + sa;
-        p.partials[(static_cast<int64_t>(un.b * p.h_q + j) * p.S + un.s) * C::kRec + kRecPad + dd] = a;
-      }
-      workers_sync<D>();          // scratch read before the next unit reuses it
-    }
-    if (bad && !kDump && widx == 0 && lane < kN) {
-      // this unit and every later one of this CTA: poisoned records
-      for (; u < n_units; u += gridDim.x) {
-        Unit un;
-        if (!unit_at(p, u, false, un) || lane >= G) continue;
-        const int j = un.kh * G + lane;
-        put_poison(p.partials + (static_cast<int64_t>(un.b * p.h_q + j) * p.S + un.s) * C::kRec);
+        workers_sync<D>();
       }
     }
   }
@@ -742,7 +526,7 @@ int sm_count(int dev) {
 
 template <int D, int MODE, bool FS>
 cudaError_t launch_tc(const StepParams &p, const CUtensorMap &kmap, const CUtensorMap &qmap,
-                      const HeadMap &hm, int dev, cudaStream_t st) {
+                      int dev, cudaStream_t st) {
   using Lo = Layout<D>;
   static std::atomic<bool> attr_set[kMaxDevices];
   if (!attr_set[dev].load(std::memory_order_acquire)) {
@@ -757,37 +541,14 @@ cudaError_t launch_tc(const StepParams &p, const CUtensorMap &kmap, const CUtens
   const int grid = n_units < sms ? n_units : sms;
   if (grid < 1) return cudaSuccess;
   return launch_pdl(saga_tc_kernel<D, MODE, FS>, dim3(grid), dim3(Cfg<D>::kThreads), Lo::alloc,
-                    st, p, kmap, qmap, hm);
-}
-
-// Lane-group slots: value head slot vs = v / chunks, chunk c = v % chunks of
-// that value head's h_q / h_v query heads (four per chunk).
-bool make_head_map(int h_q, int h_k, int h_v, HeadMap &hm) {
-  if (h_k < 1 || h_v < 1 || h_q % h_v != 0 || h_v % h_k != 0) return false;
-  const int G = h_q / h_k, hpv = h_q / h_v, vpg = h_v / h_k;
-  const int chunks = (hpv + 3) / 4;
-  if (G > kN || vpg * chunks > 4) return false;
-  for (int v = 0; v < 4; ++v) {
-    const int vs = v / chunks, c = v % chunks;
-    if (vs < vpg && c * 4 < hpv) {
-      hm.hbase[v] = vs * hpv + c * 4;
-      hm.nh[v] = hpv - c * 4 < 4 ? hpv - c * 4 : 4;
-      hm.vs[v] = vs;
-    } else {
-      hm.hbase[v] = 0;
-      hm.nh[v] = 0;
-      hm.vs[v] = 0;
-    }
-    hm.smask[v] = ((1u << hm.nh[v]) - 1u) << hm.hbase[v];
-  }
-  return true;
+                    st, p, kmap, qmap);
 }
 
 }  // namespace
 
 bool saga_tc_supports(int dtype, int d, int h_q, int h_k, int h_v) {
-  HeadMap hm;
-  return dtype == SAGA_BF16 && (d == 64 || d == 128) && make_head_map(h_q, h_k, h_v, hm);
+  return dtype == SAGA_BF16 && (d == 64 || d == 128) && h_k >= 1 && h_v >= 1 &&
+         h_q % h_v == 0 && h_v % h_k == 0 && h_q / h_k <= kN;
 }
 
 bool saga_tc_scores_streamable(const float *rows, int64_t row_stride) {
@@ -796,8 +557,7 @@ bool saga_tc_scores_streamable(const float *rows, int64_t row_stride) {
 }
 
 cudaError_t launch_saga_tc(const StepParams &p, int mode, int d, cudaStream_t st) {
-  HeadMap hm;
-  if (!make_head_map(p.h_q, p.h_k, p.h_v, hm)) return cudaErrorInvalidValue;
+  if (!saga_tc_supports(SAGA_BF16, d, p.h_q, p.h_k, p.h_v)) return cudaErrorInvalidValue;
   if (mode != kModeDump && mode != kModeStep && mode != kModeStepTies) return cudaErrorInvalidValue;
   const bool fs = p.scores_in != nullptr;
   if (fs && (mode == kModeDump || !saga_tc_scores_streamable(p.scores_in, p.row_stride)))
@@ -849,12 +609,12 @@ cudaError_t launch_saga_tc(const StepParams &p, int mode, int d, cudaStream_t st
   }
 #define SAGA_TC_LAUNCH(DD)                                                                    \
   if (d == DD) {                                                                              \
-    if (mode == kModeDump) return launch_tc<DD, kModeDump, false>(p, kmap, qmap, hm, dev, st); \
+    if (mode == kModeDump) return launch_tc<DD, kModeDump, false>(p, kmap, qmap, dev, st); \
     if (mode == kModeStep)                                                                    \
-      return fs ? launch_tc<DD, kModeStep, true>(p, kmap, qmap, hm, dev, st)                  \
-                : launch_tc<DD, kModeStep, false>(p, kmap, qmap, hm, dev, st);                \
-    return fs ? launch_tc<DD, kModeStepTies, true>(p, kmap, qmap, hm, dev, st)                \
-              : launch_tc<DD, kModeStepTies, false>(p, kmap, qmap, hm, dev, st);              \
+      return fs ? launch_tc<DD, kModeStep, true>(p, kmap, qmap, dev, st)                  \
+                : launch_tc<DD, kModeStep, false>(p, kmap, qmap, dev, st);                \
+    return fs ? launch_tc<DD, kModeStepTies, true>(p, kmap, qmap, dev, st)                \
+              : launch_tc<DD, kModeStepTies, false>(p, kmap, qmap, dev, st);              \
   }
   SAGA_TC_LAUNCH(64)
   SAGA_TC_LAUNCH(128)

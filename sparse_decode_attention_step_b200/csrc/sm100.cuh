@@ -142,6 +142,13 @@ __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
                : "memory");
 }
 
+// 4-byte asynchronous copy global -> shared through L1 (cp.async).
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)),
+               "l"(reinterpret_cast<uint64_t>(src))
+               : "memory");
+}
+
 // Close this thread's group of cp.async copies issued since the last commit.
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");

@@ -23,18 +23,24 @@ def dev(a):
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
 
 
-def planned_scratch_bytes(B, h_q, h_k, d, L):
-    """Scratch of a plain step on the tensor-core path: the 256-byte error
-    word and one (m, l, count, pad, acc[d]) float record per (b, j, split),
-    with the persistent plan's split count (148 SMs, up to 128 tiles of 128
-    positions per unit), rounded up to 256 bytes."""
-    rows = B * h_k
-    tiles = rows * -(-L // 128)
-    waves = max(1, -(-tiles // (148 * 128)))
-    s_target = max(1, 148 * waves // rows)
-    split_len = -(-(-(-L // s_target)) // 128) * 128
-    S = -(-L // split_len)
-    return -(-(256 + B * h_q * S * (d + 4) * 4) // 256) * 256
+def planned_scratch_bytes(B, h_q, h_k, h_v, d, L):
+    """Scratch of a plain step on the tensor-core path, as the library plans
+    it: the 256-byte error and abort words; one (m, l, count, pad, acc[d])
+    float record per (b, j, gather split); and, per (b, j) and 32-position
+    block, a 4-byte kept mask and 32 4-byte kept scores. Each part is rounded
+    up to 256 bytes. The gather splits each (b, j) row so that all rows take
+    at most 888 CTAs (more only when there are more rows), each at least 8
+    blocks long."""
+    up = lambda x: -(-x // 256) * 256
+    cdiv = lambda a, b: -(-a // b)
+    nblk = cdiv(L, 32)
+    sb = min(max(1, nblk // 8), max(1, 888 // (B * h_q)))
+    bps = cdiv(nblk, sb)
+    SB = cdiv(nblk, bps)
+    lists = B * h_q * nblk
+    off = up(256 + B * h_q * SB * (d + 4) * 4)
+    off = up(off + lists * 4)
+    return up(off + lists * 32 * 4)
 
 
 def test_noalloc_matches_workspace_step_twice():
@@ -77,15 +83,15 @@ def test_noalloc_matches_workspace_step_twice():
 
 
 def test_noalloc_scratch_limit_both_sides():
-    """963 sequences of 128 positions (h_q=16, h_k=2, d=64: one split per
-    sequence) need 4,191,232 bytes of scratch and run; 964 need 4,195,584,
-    more than the 4 MiB array, and are refused before anything runs."""
+    """The largest batch of 128-position sequences (h_q=16, h_k=2, h_v=4,
+    d=64) whose scratch fits the 4 MiB array runs and matches
+    saga_decode_step; one sequence more is refused before anything runs."""
     lib = saga.load()
     limit = saga.NOALLOC_SCRATCH_BYTES
     L, h_q, h_k, h_v, d = 128, 16, 2, 4, 64
-    under, over = 963, 964
-    assert planned_scratch_bytes(under, h_q, h_k, d, L) <= limit
-    assert planned_scratch_bytes(over, h_q, h_k, d, L) > limit
+    under = max(B for B in range(1, 4096) if planned_scratch_bytes(B, h_q, h_k, h_v, d, L) <= limit)
+    over = under + 1
+    assert planned_scratch_bytes(over, h_q, h_k, h_v, d, L) > limit
 
     big = saga.shape(over, h_q, h_k, h_v, d, synth.BF16, L)
     fake = 1 << 40          # never dereferenced: the call is refused first
