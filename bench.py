@@ -7,20 +7,29 @@ The default workload is the Llama-3.2-1B-shaped 16-layer stack at batch 8 and
 128K context (h_q=32, h_k=2, h_v=8, d=64, bf16 caches, N=2048, R=32).
 
 Prints one JSON line (rank 0):
-  value      steps/s of the whole job, inputs resident in HBM (CUDA events
-             over exactly --steps steps, max over ranks);
-  e2e        the same metric with queries copied in from pinned host memory
-             and outputs read back every step;
+  value      the R-cycle average of the whole job in steps/s:
+             R / (t_refresh + (R - 1) t_plain), t_plain and t_refresh the
+             medians over at least ten replays of CUDA graphs of consecutive
+             plain and consecutive refresh steps (CUDA events on the launching
+             stream, max over ranks), inputs resident in HBM; both parts are
+             in step_times. timed_steps: exactly --steps steps of the real
+             schedule (refresh at t mod R == 0, t from 0) in one graph.
+  e2e        the same metric with each step's queries copied in from pinned
+             host memory and its outputs read back;
   roofline   the plain-step call (the dominant one): algorithmic bytes per
-             call / its mean duration, against the measured HBM copy peak;
+             call / its median duration, against the measured HBM copy peak;
   dense_gqa  the library's dense GQA stack at the same shape, same metric;
   saga_full  full attention over the same SAGA-headed caches (the ablation arm
              between dense GQA and SAGA + Atop-N);
-  cpu_baseline  the float64 oracle on the host cores, on a bounded sample.
+  cpu_baseline  the float64 oracle on the host cores, on a bounded sample;
+  workloads  the same figures for the other workloads (the Qwen2.5-1.5B- and
+             Llama-3.2-1B-shaped single layers, the ragged refresh-every-step
+             batch at each N, the tiny fp32 case), unless --primary-only.
 
 With --impl reference the oracle alone is timed (the reference arm).
-Multi-GPU (torchrun): every rank runs its own batch (weak scaling), no
-collective on the data path.
+--gpus N starts N ranks (torch.distributed.run) unless already launched by
+it; every rank runs its own batch of the same workload (weak scaling), with
+no collective on the data path.
 """
 import argparse
 import hashlib
@@ -28,6 +37,7 @@ import json
 import math
 import os
 import re
+import socket
 import subprocess
 import sys
 import tempfile
@@ -41,33 +51,57 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 DEFAULT_WORKLOAD = "llama1b_stack16_b8_128k"
+EXTRA_WORKLOADS = ("qwen1p5b_128k", "llama1b_32k", "ragged_refresh_b16", "tiny_f32")
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
+MIN_REPLAYS = 10
 METRIC = "SAGA+Atop-N decode-attn steps/s at 128K ctx; HBM GB/s vs peak"
+PAGES_CONTEXT = ("the SAGA paper reports an end-to-end decode speedup above 2x over "
+                 "full-attention GQA at 128K context on Llama 3.2-1B and Qwen2.5-1.5B "
+                 "(model level, hardware not tied to the figure); its key-head merge "
+                 "alone gives up to 1.47x at batch 16 and 128K")
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=64)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
-    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--primary-only", action="store_true",
+                    help="measure the --workload alone, without the other workloads")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--dense-steps", type=int, default=8)
     ap.add_argument("--layers", type=int, default=None,
                     help="override the stack depth (same per-layer launch, smaller footprint)")
     ap.add_argument("--merge", default=None,
                     help="time the closed-form GQA-to-SAGA key merge on this calibration "
                          "workload instead (synth.merge_workload.MERGE_WORKLOADS)")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 # ---------------------------------------------------------------------------
 # distributed plumbing
 # ---------------------------------------------------------------------------
+def free_port():
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def spawn_ranks(args, argv):
+    """--gpus N > 1 outside torch.distributed.run: start N ranks through it
+    (one process per GPU, rendezvous on 127.0.0.1) and return their exit
+    status; None when this process is a rank already or N == 1."""
+    if args.gpus <= 1 or "WORLD_SIZE" in os.environ:
+        return None
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={args.gpus}", "--master-addr=127.0.0.1",
+           f"--master-port={free_port()}", os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
+
+
 def dist_init(backend=None):
     """One process per GPU: NCCL over the node's GPUs (gloo for CPU-only
     checks). Returns (world, rank, local_rank)."""
@@ -114,6 +148,13 @@ def sum_over_ranks(x, world):
     return _reduce(x, world, dist.ReduceOp.SUM if world > 1 else None)
 
 
+def finish_dist(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def rank_workload(w, rank):
     """Each rank decodes its own batch of the same workload (weak scaling):
     rank 0 keeps the canonical seed, rank r > 0 draws independent inputs."""
@@ -124,6 +165,17 @@ def aggregate_value(steps, max_ms, world):
     """Whole-job steps/s: every rank ran `steps` steps of its own batch; the
     job takes as long as the slowest rank."""
     return world * steps / (max_ms / 1e3)
+
+
+def r_cycle(t_plain_ms, t_refresh_ms, R):
+    """Steps/s of one rank averaged over a refresh cycle of R steps: one
+    refresh step and R - 1 plain steps."""
+    return R / ((t_refresh_ms + (R - 1) * t_plain_ms) / 1e3)
+
+
+def step_schedule(n, R):
+    """Refresh flags of steps 0 .. n-1 (t mod R == 0)."""
+    return [t % R == 0 for t in range(n)]
 
 
 # ---------------------------------------------------------------------------
@@ -212,7 +264,7 @@ def step_kernel_sources():
     """The sources the decode step's kernels and plan are built from."""
     here = os.path.join(ROOT, "sparse_decode_attention_step_b200", "csrc")
     return [os.path.join(here, f) for f in ("common.cuh", "sm100.cuh", "kernels.h",
-                                            "saga_api.cu", "saga_tc.cu", "combine.cu")]
+                                            "saga_api.cu", "saga_tc.cu", "gather.cu", "combine.cu")]
 
 
 def ncu_traffic(kernel_sources):
@@ -234,7 +286,7 @@ class OracleSample:
     """One (sequence, key-head group) of one layer, the bounded sample the
     oracle is timed on; scaled by the number of such groups per step."""
 
-    def __init__(self, w):
+    def __init__(self, w, steps=2):
         self.w = w
         L = int(synth.seq_lens(w)[0])
         G = w.h_q // w.h_k
@@ -246,9 +298,7 @@ class OracleSample:
         self.K = K[None, None]             # [1][1][L][d]
         self.V = V[None]                   # [1][hv_g][L][d]
         self.l = np.array([L])
-        steps = max(2, 2)
-        qs = synth.widen(synth.queries(w, 0, steps, B=1, h_q=G))
-        self.qs = qs                       # [steps][1][G][d]
+        self.qs = synth.widen(synth.queries(w, 0, max(2, steps), B=1, h_q=G))   # [steps][1][G][d]
         self.tau = None
 
     def step(self, t, refresh):
@@ -270,7 +320,7 @@ def blas_threads():
 
 def time_oracle(w, n_plain=2, n_refresh=1):
     """Seconds per full step (every layer, sequence and key-head group), from
-    timing the sample's plain and refresh steps."""
+    timing the sample's plain and refresh steps, averaged over a refresh cycle."""
     s = OracleSample(w)
     s.step(0, True)                                   # warm
     t0 = time.perf_counter()
@@ -285,17 +335,39 @@ def time_oracle(w, n_plain=2, n_refresh=1):
     return per_group * s.groups_per_step, t_plain, t_ref, s
 
 
+def cpu_baseline_entry(w):
+    step_s, t_plain, t_ref, s = time_oracle(w)
+    return {"value": 1.0 / step_s, "unit": "steps/s", "cores": os.cpu_count(),
+            "blas_threads": blas_threads(), "kind": "oracle",
+            "sample": (f"layer 0, sequence 0, key head 0 ({s.G} query heads, l_kv={s.L}): "
+                       f"1 refresh + 2 plain steps timed, R-cycle average, scaled by "
+                       f"{s.groups_per_step} groups per step"),
+            "sample_plain_s": t_plain, "sample_refresh_s": t_ref}
+
+
+def workload_config(w, world, replicas=1):
+    return {"workload": w.name, "batch_per_gpu": w.B, "global_batch": w.B * world,
+            "layers": w.layers, "h_q": w.h_q, "h_k": w.h_k, "h_v": w.h_v, "d": w.d,
+            "l_kv": w.l_kv if w.l_kv_range is None else list(w.l_kv_range), "N": w.N,
+            "R": w.R, "dense_gqa_h_kv": w.dense_hkv,
+            "parallelism": f"weak: {world} independent batch replica(s)",
+            "l2": ("inputs larger than L2" if replicas == 1 else
+                   f"{replicas} bit-identical cache replicas rotated"),
+            "timed_region": ("CUDA graphs of consecutive steps of one kind (R-cycle value); "
+                             "the --steps schedule in one graph (timed_steps)")}
+
+
 def reference_arm(args, w):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
-        return
-    s = OracleSample(w)
+        return                     # rank 0 alone times the oracle; no process group
+    s = OracleSample(w, steps=args.warmup + args.steps)
     for t in range(args.warmup):
         s.step(t, t % w.R == 0)
     t0 = time.perf_counter()
-    for t in range(args.warmup, args.warmup + args.steps):
-        s.step(t, t % w.R == 0)
+    for t in range(args.steps):
+        s.step(args.warmup + t, t % w.R == 0)
     sample_s = time.perf_counter() - t0
     step_s = sample_s / args.steps * s.groups_per_step
     v = 1.0 / step_s
@@ -306,26 +378,34 @@ def reference_arm(args, w):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(w, world),
-        "cpu_baseline": {"value": v, "unit": "steps/s", "cores": blas_threads(),
-                         "kind": "oracle", "sample": sample},
+        "config": workload_config(w, world, replicas_for(w)),
+        "cpu_baseline": {"value": v, "unit": "steps/s", "cores": os.cpu_count(),
+                         "blas_threads": blas_threads(), "kind": "oracle", "sample": sample},
         "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
-def workload_config(w, world):
-    return {"workload": w.name, "batch_per_gpu": w.B, "global_batch": w.B * world,
-            "layers": w.layers, "h_q": w.h_q, "h_k": w.h_k, "h_v": w.h_v, "d": w.d,
-            "l_kv": w.l_kv if w.l_kv_range is None else list(w.l_kv_range), "N": w.N,
-            "R": w.R, "dense_gqa_h_kv": w.dense_hkv,
-            "parallelism": f"weak: {world} independent batch replica(s)"}
-
-
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
+def stack_cap(w):
+    """Cache capacity: the longest sequence rounded up to 128 positions."""
+    return int(math.ceil(int(synth.seq_lens(w).max()) / 128) * 128)
+
+
+def replicas_for(w, dense=False):
+    """Single-layer workloads rotate bit-identical cache replicas so the
+    working set stays well above L2."""
+    if w.layers > 1:
+        return 1
+    h = w.dense_hkv if dense else w.h_k
+    hv = w.dense_hkv if dense else w.h_v
+    layer_bytes = w.B * (h + hv) * stack_cap(w) * w.d * w.elem_bytes
+    return max(1, math.ceil(4 * L2_BYTES / layer_bytes))
+
+
 class Stack:
     """Device state of one attention stack: per-layer caches, thresholds,
     outputs, the static query buffer and the workspace."""
@@ -338,14 +418,10 @@ class Stack:
         h_v = w.dense_hkv if dense else w.h_v
         kk, vk = ("KD", "VD") if dense else ("K", "V")
         self.lens = synth.seq_lens(w)
-        cap = int(self.lens.max())
+        cap = stack_cap(w)
         self.cap = cap
         self.shape = saga.shape(w.B, w.h_q, h_k, h_v, w.d, w.dtype, cap, cap)
-        esz = w.elem_bytes
-        layer_bytes = w.B * (h_k + h_v) * cap * w.d * esz
-        # single-layer workloads rotate bit-identical replicas so the working
-        # set stays well above L2
-        self.replicas = 1 if w.layers > 1 else max(1, math.ceil(4 * L2_BYTES / layer_bytes))
+        self.replicas = replicas_for(w, dense)
         self.nl = w.layers
         dt = torch.float32 if w.dtype == synth.F32 else torch.int16
         self.K, self.V = [], []
@@ -368,22 +444,22 @@ class Stack:
         self.ws = saga.Workspace(self.shape, w.N)
         self.saga = saga
 
-    def layer_call(self, t, l, refresh, sel_mask=None):
+    def layer_call(self, t, l, refresh, sel_mask=None, N=None):
         r = t % self.replicas
         K, V = self.K[r * self.nl + l], self.V[r * self.nl + l]
         s = self.saga
         if self.dense:
             s.gqa_dense_decode(self.shape, self.q[l], K, V, self.l, self.out[l], self.ws)
         elif refresh:
-            s.refresh_threshold(self.shape, self.q[l], K, self.l, self.w.N, self.tau[l], self.ws,
-                                V=V, out=self.out[l], sel_mask=sel_mask)
+            s.refresh_threshold(self.shape, self.q[l], K, self.l, self.w.N if N is None else N,
+                                self.tau[l], self.ws, V=V, out=self.out[l], sel_mask=sel_mask)
         else:
             s.decode_step(self.shape, self.q[l], K, V, self.l, self.tau[l], self.out[l], self.ws,
                           sel_mask=sel_mask)
 
-    def step(self, t, refresh):
+    def step(self, t, refresh, N=None):
         for l in range(self.nl):
-            self.layer_call(t, l, refresh)
+            self.layer_call(t, l, refresh, N=N)
 
     def full_step(self, t):
         """Full attention over the same (SAGA-headed) caches, every layer."""
@@ -392,11 +468,256 @@ class Stack:
             self.saga.dense_decode(self.shape, self.q[l], self.K[r * self.nl + l],
                                    self.V[r * self.nl + l], self.l, self.out[l], self.ws)
 
+    def free(self):
+        import torch
+        self.K, self.V = [], []
+        torch.cuda.empty_cache()
+
 
 def kernels_per_call(dense, refresh):
     if dense:
         return 2                  # dense split + combine
-    return 4 if refresh else 2    # (dump, radix,) split + combine
+    return 4 if refresh else 2    # (dump, radix,) step + combine
+
+
+def graph_of(fn):
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
+
+
+def replay_ms(g, n, stream):
+    """Device time of each of n back-to-back replays of graph g (CUDA events
+    on the launching stream; the host is kept ahead of the GPU)."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n)]
+    torch.cuda.synchronize()
+    torch.cuda._sleep(int(2e7))
+    for a, b in evs:
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def call_ms(fn, n, stream):
+    """Device time of each of n direct calls of fn (host kept ahead)."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n)]
+    torch.cuda.synchronize()
+    torch.cuda._sleep(int(2e8))
+    for i, (a, b) in enumerate(evs):
+        a.record(stream)
+        fn(i)
+        b.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def measure_saga(w, args, saga, world, rank, N=None, st=None, with_dense=True, with_cpu=True):
+    """All figures of one workload (and one N): the R-cycle value and its
+    parts, the --steps schedule, e2e, roofline, dense GQA, SAGA full
+    attention and the CPU baseline. Returns (dict, stack)."""
+    import torch
+    N = w.N if N is None else N
+    R, nl = w.R, w.layers
+    own = st is None
+    if own:
+        st = Stack(w, saga)
+    esz = w.elem_bytes
+    reps = 4 if nl > 1 else 32                     # steps per graph replay
+    W, K = max(3, args.warmup), args.steps
+    n_q = W + K + 2 * reps
+    qh = np.stack([synth.queries(w, l, n_q) for l in range(nl)], axis=1)
+    if w.dtype != synth.F32:
+        qh = qh.view(np.int16)
+    Q = torch.from_numpy(qh).cuda()                # [step][layer][B][h_q][d]
+    Qpin = torch.from_numpy(qh).pin_memory()
+    stream = torch.cuda.current_stream()
+    sched = step_schedule(K, R)
+
+    def run_steps(idx0, n, kind):
+        # n steps with queries idx0.., refresh by `kind` (a list of flags or a bool)
+        for i in range(n):
+            st.q.copy_(Q[idx0 + i], non_blocking=True)
+            st.step(idx0 + i, kind[i] if isinstance(kind, list) else kind, N=N)
+
+    # warm-up: every kernel loaded and tau set before any capture
+    run_steps(0, W, step_schedule(W, R))
+    torch.cuda.synchronize()
+    g_timed = graph_of(lambda: run_steps(W, K, sched))
+    g_plain = graph_of(lambda: run_steps(W + K, reps, False))
+    g_ref = graph_of(lambda: run_steps(W + K + reps, reps, True))
+    torch.cuda.synchronize()
+    barrier(world)
+
+    # ---- the --steps schedule, then the R-cycle parts ---------------------
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda._sleep(int(2e7))
+    ev0.record(stream)
+    g_timed.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    timed_ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+    n_plain = max(MIN_REPLAYS, 64 // reps)
+    plain = replay_ms(g_plain, n_plain, stream) if R > 1 else []
+    refr = replay_ms(g_ref, max(MIN_REPLAYS, 16 // reps), stream)
+    t_plain = max_over_ranks(float(np.median(plain)) / reps, world) if plain else None
+    t_ref = max_over_ranks(float(np.median(refr)) / reps, world)
+    per_rank = r_cycle(t_plain, t_ref, R) if R > 1 else 1e3 / t_ref
+    value = world * per_rank
+    n_refresh = sum(sched)
+    launches = nl * (n_refresh * kernels_per_call(False, True)
+                     + (K - n_refresh) * kernels_per_call(False, False))
+    del g_timed, g_plain, g_ref
+
+    # ---- roofline of the dominant call: the plain step (the refresh at R = 1)
+    dom_refresh = R == 1
+    n_calls = 24
+
+    def one_call(i):
+        st.q.copy_(Q[W + K + i % (2 * reps)])
+        st.layer_call(i, i % nl, dom_refresh, N=N)
+    ms = call_ms(one_call, n_calls, stream)
+    call = float(np.median(ms))
+    B, h_q, h_k, h_v, d = w.B, w.h_q, w.h_k, w.h_v, w.d
+    lens = st.lens.astype(np.int64)
+    k_bytes = float(np.sum(h_k * lens * d * esz))
+    qo_bytes = B * h_q * d * (esz + 4) + B * h_q * 4
+    mask = torch.zeros(B, h_q, st.cap, dtype=torch.uint8, device="cuda")
+    v_bytes, v_nodedup = [], []
+    for i in range(4):
+        st.q.copy_(Q[W + K + i])
+        mask.zero_()
+        st.layer_call(i, i % nl, dom_refresh, sel_mask=mask, N=N)
+        m = mask.view(B, h_v, h_q // h_v, st.cap)
+        v_bytes.append(int(m.amax(dim=2).sum().item()) * d * esz)
+        v_nodedup.append(int(mask.sum().item()) * d * esz)
+    torch.cuda.synchronize()
+    del mask
+    alg = k_bytes + float(np.mean(v_bytes)) + qo_bytes
+    peak, peak_kind = measured_peaks()
+    achieved = alg / (call / 1e3) / 1e9
+    roof = {"bound": "hbm",
+            "kernel": ("saga_refresh_threshold (score pass, select, stored-score step, combine)"
+                       if dom_refresh else "saga_decode_step (step kernel + combine)"),
+            "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+            "peak_source": peak_kind,
+            "traffic": None if dom_refresh else ncu_traffic(step_kernel_sources()),
+            "alg_bytes_per_call": alg, "call_ms": call, "calls_timed": n_calls,
+            "v_bytes_per_call_distinct": float(np.mean(v_bytes)),
+            "v_bytes_per_call_nodedup": float(np.mean(v_nodedup)),
+            "frac_of_8000_nominal": achieved / 8000.0}
+
+    # ---- e2e: each step's queries in from pinned host memory, outputs back
+    out_pin = torch.empty(st.out.shape, dtype=torch.float32).pin_memory()
+    l_pin = torch.from_numpy(st.lens).pin_memory()
+    g1 = {}
+    for r in range(st.replicas):
+        for kind in ((True, False) if R > 1 else (True,)):
+            g1[(kind, r)] = graph_of(lambda r=r, kind=kind: st.step(r, kind, N=N))
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e = {True: [], False: []}
+    n_e2e = MIN_REPLAYS + 2
+    for kind in g1and_kinds(R):
+        for i in range(n_e2e):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            st.q.copy_(Qpin[W + K + i % (2 * reps)], non_blocking=True)
+            st.l.copy_(l_pin, non_blocking=True)
+            g1[(kind, i % st.replicas)].replay()
+            out_pin.copy_(st.out, non_blocking=True)
+            b.record(stream)
+            stream.synchronize()
+            e2e[kind].append(a.elapsed_time(b))
+    e2e_p = max_over_ranks(float(np.median(e2e[False])), world) if R > 1 else None
+    e2e_f = max_over_ranks(float(np.median(e2e[True])), world)
+    e2e_value = world * (r_cycle(e2e_p, e2e_f, R) if R > 1 else 1e3 / e2e_f)
+    h2d = Q[0].numel() * Q.element_size() + l_pin.numel() * 4
+    d2h = st.out.numel() * 4
+    del g1
+
+    res = {
+        "value": value, "unit": "steps/s", "ms_per_step": 1e3 / value * world,
+        "tokens_per_s": value * B,
+        "step_times": {"plain_ms": t_plain, "refresh_ms": t_ref, "refresh_every": R,
+                       "steps_per_replay": reps, "replays": [len(plain), len(refr)],
+                       "statistic": "median per step, max over ranks"},
+        "timed_steps": {"steps": K, "refresh_steps": n_refresh, "ms": timed_ms,
+                        "steps_per_s": aggregate_value(K, timed_ms, world)},
+        "gpu_launches": launches * world,
+        "roofline": roof,
+        "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "plain_ms": e2e_p, "refresh_ms": e2e_f},
+        "N": N,
+    }
+
+    # ---- dense GQA stack at the same shape, and SAGA full attention --------
+    if with_dense and not args.no_dense and w.dense_hkv is not None:
+        dst = Stack(w, saga, dense=True)
+        dst.q.copy_(Q[0])
+        dst.step(0, False)
+        torch.cuda.synchronize()
+        dreps = 2 if nl > 1 else 16
+
+        def dense_steps():
+            for i in range(dreps):
+                dst.q.copy_(Q[i], non_blocking=True)
+                dst.step(i, False)
+        gd = graph_of(dense_steps)
+        dms = max_over_ranks(float(np.median(replay_ms(gd, MIN_REPLAYS, stream))) / dreps, world)
+        del gd
+        dbytes = nl * (2 * w.dense_hkv * float(np.sum(lens)) * d * esz + qo_bytes)
+        dgbs = dbytes / (dms / 1e3) / 1e9
+        dvalue = world * 1e3 / dms
+        res["dense_gqa"] = {"value": dvalue, "unit": "steps/s", "ms_per_step": dms,
+                            "tokens_per_s": dvalue * B, "achieved_gbs": dgbs,
+                            "frac_of_peak": dgbs / peak, "h_kv": w.dense_hkv,
+                            "speedup_saga_over_dense": value / dvalue}
+        dst.free()
+        del dst
+    if with_dense and not args.no_dense and w.h_k != w.h_v:
+        freps = 2 if nl > 1 else 16
+
+        def full_steps():
+            for i in range(freps):
+                st.q.copy_(Q[i], non_blocking=True)
+                st.full_step(i)
+        full_steps()
+        torch.cuda.synchronize()
+        gf = graph_of(full_steps)
+        fms = max_over_ranks(float(np.median(replay_ms(gf, MIN_REPLAYS, stream))) / freps, world)
+        del gf
+        fbytes = nl * ((w.h_k + w.h_v) * float(np.sum(lens)) * d * esz + qo_bytes)
+        fgbs = fbytes / (fms / 1e3) / 1e9
+        fvalue = world * 1e3 / fms
+        res["saga_full"] = {"value": fvalue, "unit": "steps/s", "ms_per_step": fms,
+                            "tokens_per_s": fvalue * B, "achieved_gbs": fgbs,
+                            "frac_of_peak": fgbs / peak, "h_k": w.h_k, "h_v": w.h_v,
+                            "speedup_saga_atopn_over_full": value / fvalue}
+        if "dense_gqa" in res:
+            res["saga_full"]["speedup_full_over_dense_gqa"] = fvalue / res["dense_gqa"]["value"]
+    if with_cpu and rank == 0 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline_entry(w.with_(N=N))
+    res["config"] = workload_config(w, world, st.replicas)
+    res["config"]["N"] = N
+    del Q, Qpin
+    if own:
+        st.free()
+    return res, (None if own else st)
+
+
+def g1and_kinds(R):
+    return (True, False) if R > 1 else (True,)
 
 
 def run_ours(args, w):
@@ -404,274 +725,45 @@ def run_ours(args, w):
     import sparse_decode_attention_step_b200 as saga
     saga.load()
     world, rank, local = dist_init()
-    w = rank_workload(w, rank)
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but {world} ranks were started")
     torch.manual_seed(0)
-    R = w.R
-    T_total = args.warmup + args.steps
-    st = Stack(w, saga)
-    esz = w.elem_bytes
-    # queries of every step, resident in HBM, and their pinned host copies
-    qh = np.stack([synth.queries(w, l, T_total) for l in range(w.layers)], axis=1)
-    if w.dtype != synth.F32:
-        qh = qh.view(np.int16)
-    Q = torch.from_numpy(qh).cuda()                     # [T][layers][B][h_q][d]
-    Qpin = torch.from_numpy(qh).pin_memory()
-    torch.cuda.synchronize()
-
-    stream = torch.cuda.current_stream()
-
-    def enqueue(t):
-        st.q.copy_(Q[t], non_blocking=True)
-        st.step(t, t % R == 0)
-
-    def capture(t0, t1):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            for t in range(t0, t1):
-                enqueue(t)
-        return g
-
-    # warm-up steps run directly (they load every kernel before any capture)
-    for t in range(args.warmup):
-        enqueue(t)
-    torch.cuda.synchronize()
-    use_graph = not args.no_graph
-    if use_graph:
-        g_timed = capture(args.warmup, T_total)
-        torch.cuda.synchronize()
-    barrier(world)
-
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    names = [w.name] + ([] if args.primary_only else [n for n in EXTRA_WORKLOADS if n != w.name])
+    results = {}
     with ClockSampler(local) as clk:
-        time.sleep(0.3)
-        torch.cuda.synchronize()
-        barrier(world)
-        if not use_graph:
-            torch.cuda._sleep(int(2e8))      # let the host run ahead of the GPU
-        ev0.record(stream)
-        if use_graph:
-            g_timed.replay()
-        else:
-            for t in range(args.warmup, T_total):
-                enqueue(t)
-        ev1.record(stream)
-        torch.cuda.synchronize()
-        barrier(world)
-    elapsed_ms = ev0.elapsed_time(ev1)
-    max_ms = max_over_ranks(elapsed_ms, world)
-    value = aggregate_value(args.steps, max_ms, world)
-    n_refresh = sum(1 for t in range(args.warmup, T_total) if t % R == 0)
-    launches = w.layers * (n_refresh * kernels_per_call(False, True)
-                           + (args.steps - n_refresh) * kernels_per_call(False, False))
-    if use_graph:
-        del g_timed
-
-    # ---- roofline: per-call durations of plain steps, and algorithmic bytes
-    # from a validation pass with the selection dumped
-    torch.cuda.synchronize()
-    evs = []
-    n_rl = min(args.steps, 2 * R)
-    torch.cuda._sleep(int(4e8))              # let the host run ahead of the GPU
-    for t in range(args.warmup, args.warmup + n_rl):
-        st.q.copy_(Q[t])
-        refresh = t % R == 0
-        for l in range(w.layers):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            st.layer_call(t, l, refresh)
-            b.record(stream)
-            evs.append((refresh, a, b))
-    torch.cuda.synchronize()
-    plain_ms = [a.elapsed_time(b) for (r, a, b) in evs if not r]
-    refresh_ms = [a.elapsed_time(b) for (r, a, b) in evs if r]
-    call_ms = float(np.mean(plain_ms)) if plain_ms else float("nan")
-    refresh_call_ms = float(np.mean(refresh_ms)) if refresh_ms else None
-
-    B, h_q, h_k, h_v, d = w.B, w.h_q, w.h_k, w.h_v, w.d
-    lens = st.lens.astype(np.int64)
-    k_bytes = float(np.sum(h_k * lens * d * esz))
-    qo_bytes = B * h_q * d * (esz + 4) + B * h_q * 4
-    mask = torch.zeros(B, h_q, st.cap, dtype=torch.uint8, device="cuda")
-    v_bytes, v_bytes_nodedup = [], []
-    for t in range(args.warmup, args.warmup + min(args.steps, 2 * R)):
-        st.q.copy_(Q[t])
-        refresh = t % R == 0
-        for l in range(w.layers):
-            mask.zero_()
-            st.layer_call(t, l, refresh, sel_mask=mask)
-            if refresh:
-                continue
-            m = mask.view(B, h_v, h_q // h_v, st.cap)
-            distinct = int(m.amax(dim=2).sum().item())
-            v_bytes.append(distinct * d * esz)
-            v_bytes_nodedup.append(int(mask.sum().item()) * d * esz)
-    torch.cuda.synchronize()
-    alg_bytes = k_bytes + float(np.mean(v_bytes)) + qo_bytes
-    achieved = alg_bytes / (call_ms / 1e3) / 1e9
-    peak, peak_kind = measured_peaks()
-    traffic = ncu_traffic(step_kernel_sources())
-
-    # ---- e2e: queries in from pinned host memory, outputs back, every step
-    out_pin = torch.empty(st.out.shape, dtype=torch.float32).pin_memory()
-    l_pin = torch.from_numpy(st.lens).pin_memory()
-    graphs = {}
-    if use_graph:
-        for r in range(st.replicas):
-            for kind in (True, False):
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g):
-                    st.step(r, kind)
-                graphs[(kind, r)] = g
-    torch.cuda.synchronize()
-    barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for t in range(args.warmup, T_total):
-        st.q.copy_(Qpin[t], non_blocking=True)
-        st.l.copy_(l_pin, non_blocking=True)
-        refresh = t % R == 0
-        if graphs:
-            graphs[(refresh, t % st.replicas)].replay()
-        else:
-            st.step(t, refresh)
-        out_pin.copy_(st.out, non_blocking=True)
-        stream.synchronize()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e_value = aggregate_value(args.steps, e2e_ms, world)
-    h2d = Q[0].numel() * Q.element_size() + l_pin.numel() * 4
-    d2h = st.out.numel() * 4
-
-    # ---- dense GQA stack at the same shape
-    dense = None
-    if not args.no_dense and w.dense_hkv is not None:
-        del graphs
-        stk_dense = Stack(w, saga, dense=True)
-        stk_dense.q.copy_(Q[0])
-        for t in range(2):
-            stk_dense.step(t, False)
-        torch.cuda.synchronize()
-        barrier(world)
-        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        nd = args.dense_steps
-
-        def dense_steps():
-            for t in range(nd):
-                stk_dense.q.copy_(Q[t % T_total], non_blocking=True)
-                stk_dense.step(t, False)
-        if use_graph:
-            gd = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gd):
-                dense_steps()
-            torch.cuda.synchronize()
-        else:
-            torch.cuda._sleep(int(2e8))
-        d0.record(stream)
-        if use_graph:
-            gd.replay()
-        else:
-            dense_steps()
-        d1.record(stream)
-        torch.cuda.synchronize()
-        dms = max_over_ranks(d0.elapsed_time(d1), world)
-        dvalue = aggregate_value(nd, dms, world)
-        dbytes_step = w.layers * (2 * w.dense_hkv * float(np.sum(lens)) * d * esz + qo_bytes)
-        dgbs = dbytes_step / (dms / nd / 1e3) / 1e9
-        dense = {"value": dvalue, "unit": "steps/s", "ms_per_step": dms / nd,
-                 "tokens_per_s": dvalue * B, "achieved_gbs": dgbs, "frac_of_peak": dgbs / peak,
-                 "h_kv": w.dense_hkv, "steps": nd, "speedup_saga_over_dense": value / dvalue}
-        del stk_dense
-        torch.cuda.empty_cache()
-
-    # ---- SAGA full attention on the same stack: the ablation's "SAGA, full" arm
-    full = None
-    if not args.no_dense and w.h_k != w.h_v:
-        st.q.copy_(Q[0])
-        for t in range(2):
-            st.full_step(t)
-        torch.cuda.synchronize()
-        barrier(world)
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        nf = args.dense_steps
-
-        def full_steps():
-            for t in range(nf):
-                st.q.copy_(Q[t % T_total], non_blocking=True)
-                st.full_step(t)
-        if use_graph:
-            gf = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gf):
-                full_steps()
-            torch.cuda.synchronize()
-        else:
-            torch.cuda._sleep(int(2e8))
-        f0.record(stream)
-        if use_graph:
-            gf.replay()
-        else:
-            full_steps()
-        f1.record(stream)
-        torch.cuda.synchronize()
-        fms = max_over_ranks(f0.elapsed_time(f1), world)
-        fvalue = aggregate_value(nf, fms, world)
-        fbytes_step = w.layers * ((w.h_k + w.h_v) * float(np.sum(lens)) * d * esz + qo_bytes)
-        fgbs = fbytes_step / (fms / nf / 1e3) / 1e9
-        full = {"value": fvalue, "unit": "steps/s", "ms_per_step": fms / nf,
-                "tokens_per_s": fvalue * B, "achieved_gbs": fgbs, "frac_of_peak": fgbs / peak,
-                "h_k": w.h_k, "h_v": w.h_v, "steps": nf,
-                "speedup_saga_atopn_over_full": value / fvalue,
-                "speedup_full_over_dense_gqa": (fvalue / dense["value"]) if dense else None}
-        if use_graph:
-            del gf
-
+        for name in names:
+            ww = w if name == w.name else synth.WORKLOADS[name]
+            ww = rank_workload(ww, rank)
+            if ww.N_sweep:
+                st = Stack(ww, saga)
+                for N in ww.N_sweep:
+                    results[f"{name}_N{N}"], st = measure_saga(ww, args, saga, world, rank, N=N, st=st,
+                                                               with_dense=False)
+                st.free()
+                del st
+            else:
+                results[name], _ = measure_saga(ww, args, saga, world, rank)
+            torch.cuda.empty_cache()
     clocks = clk.summary()
-    result = None
     if rank == 0:
-        cpu = None
-        if not args.no_cpu_baseline:
-            step_s, t_plain, t_ref, s = time_oracle(w)
-            cpu = {"value": 1.0 / step_s, "unit": "steps/s", "cores": blas_threads(),
-                   "kind": "oracle",
-                   "sample": (f"layer 0, sequence 0, key head 0 ({s.G} query heads, "
-                              f"l_kv={s.L}): 1 refresh + 2 plain steps timed, R-cycle "
-                              f"average, scaled by {s.groups_per_step} groups per step"),
-                   "sample_plain_s": t_plain, "sample_refresh_s": t_ref}
-        result = {
-            "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms / args.steps,
+        primary_key = w.name if w.name in results else f"{w.name}_N{w.N}"
+        p = results.pop(primary_key)
+        line = {
+            "metric": METRIC, "value": p["value"], "unit": "steps/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": 1e3 / p["value"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if w.dtype != synth.F32 else "f32", "accumulate": "f32",
             "data": "synthetic (seeded Philox N(0,1) K/V, 1% planted keys, AR(1) queries)",
-            "config": dict(workload_config(w, world),
-                           l2="inputs larger than L2" if st.replicas == 1 else
-                           f"{st.replicas} bit-identical cache replicas rotated",
-                           timed_region="one CUDA graph of all timed steps" if use_graph
-                           else "direct launches"),
-            "tokens_per_s": value * B,
-            "refresh_every": R, "refresh_steps_timed": n_refresh,
-            "gpu_launches": launches * world,
-            "roofline": {"bound": "hbm", "kernel": "saga_decode_step (split + combine)",
-                         "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "peak_source": peak_kind,
-                         "traffic": traffic, "alg_bytes_per_call": alg_bytes,
-                         "call_ms": call_ms, "refresh_call_ms": refresh_call_ms,
-                         "v_bytes_per_call_distinct": float(np.mean(v_bytes)),
-                         "v_bytes_per_call_nodedup": float(np.mean(v_bytes_nodedup)),
-                         "frac_of_8000_nominal": achieved / 8000.0},
-            "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
-            "dense_gqa": dense,
-            "saga_full": full,
-            "clocks": clocks,
-            "cpu_baseline": cpu,
+            "config": p.pop("config"),
+            "tokens_per_s": p.pop("tokens_per_s"), "refresh_every": w.R,
         }
-        print(json.dumps(result), flush=True)
-    barrier(world)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
-    return result
+        p.pop("value"), p.pop("unit"), p.pop("ms_per_step")
+        line.update(p)
+        line["clocks"] = clocks
+        line["pages_context"] = PAGES_CONTEXT
+        line["workloads"] = results
+        print(json.dumps(line), flush=True)
+    finish_dist(world)
 
 
 # ---------------------------------------------------------------------------
@@ -778,7 +870,11 @@ def bench_merge(args):
 
 
 def main():
-    args = parse()
+    argv = sys.argv[1:]
+    args = parse(argv)
+    rc = spawn_ranks(args, argv)
+    if rc is not None:
+        sys.exit(rc)
     if args.merge is not None:
         bench_merge(args)
         return

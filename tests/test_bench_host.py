@@ -77,3 +77,29 @@ def test_aggregate_and_config(bench):
     assert cfg["workload"] == w.name and cfg["global_batch"] == 2 * w.B
     assert bench.rank_workload(w, 0) is w
     assert bench.rank_workload(w, 1).seed != w.seed
+
+
+def test_r_cycle_and_schedule(bench):
+    """The headline is the average over a refresh cycle of R steps: one
+    refresh step and R - 1 plain steps; step t refreshes when t mod R == 0."""
+    assert bench.r_cycle(1.0, 4.0, 1) == pytest.approx(1e3 / 4.0)
+    assert bench.r_cycle(1.0, 4.0, 32) == pytest.approx(32 / (4.0 + 31 * 1.0) * 1e3)
+    s = bench.step_schedule(70, 32)
+    assert [t for t, f in enumerate(s) if f] == [0, 32, 64]
+
+
+def test_config_keys_match_between_arms(bench):
+    """The reference arm and our arm report the same config keys."""
+    import synth
+    w = synth.WORKLOADS["qwen1p5b_128k"]
+    a = bench.workload_config(w, 1, bench.replicas_for(w))
+    assert {"workload", "l2", "timed_region", "N", "R", "global_batch"} <= set(a)
+    assert bench.stack_cap(synth.WORKLOADS["ragged_refresh_b16"]) % 128 == 0
+
+
+def test_spawn_only_outside_torchrun(bench, monkeypatch):
+    args = bench.parse(["--gpus", "1"])
+    assert bench.spawn_ranks(args, []) is None
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    args = bench.parse(["--gpus", "2"])
+    assert bench.spawn_ranks(args, []) is None
