@@ -227,12 +227,18 @@ saga_status saga_append_kv(const saga_shape *shape, const void *k_new,
  * softmax states) in one fixed array of SAGA_NOALLOC_SCRATCH_BYTES compiled
  * into the library; every GPU that loads the library holds that array until
  * the process exits. The paper has no counterpart to this entry point.
- *   - The step needs 256 + 4*B*h_q*S*(d+4) bytes of scratch, S being the
- *     number of l_kv splits the library plans (at most a few hundred); a
- *     shape needing more than SAGA_NOALLOC_SCRATCH_BYTES is rejected with
- *     SAGA_ERR_WORKSPACE, an invalid one with SAGA_ERR_INVALID_ARG, and
- *     nothing is enqueued then. (The 16-layer batch-8 128K workload needs
- *     about 0.6 MB per layer call.)
+ *   - On the tensor-core path the step needs, each part rounded up to 256
+ *     bytes: 256 bytes of error and abort words; 4*B*h_q*SB*(d+4) bytes of
+ *     per-split softmax states, SB being the gather splits of a (b, query
+ *     head) row the library plans (at most max_l_kv/256, and no more than
+ *     1184/(B*h_q) when that is larger than one); and 132*B*h_q*nblk bytes of
+ *     per-head kept lists, nblk = ceil(max_l_kv/32) (a 32-bit mask and 32
+ *     fp32 kept scores per 32-position block). A shape needing more than
+ *     SAGA_NOALLOC_SCRATCH_BYTES is rejected with SAGA_ERR_WORKSPACE, an
+ *     invalid one with SAGA_ERR_INVALID_ARG, and nothing is enqueued then.
+ *     (The 16-layer batch-8 128K Llama-3.2-1B workload, h_q = 32, needs
+ *     about 139 MB per layer call; batch-1 128K Qwen2.5-1.5B, h_q = 12,
+ *     about 7.1 MB.)
  *   - It calls no cudaMalloc, cudaFree or other allocating routine.
  *   - The first call on each device looks up the array's device address
  *     with that device current; make that first call before any stream
@@ -242,8 +248,13 @@ saga_status saga_append_kv(const saga_shape *shape, const void *k_new,
  *     without ordering) race on it and must be serialised by the caller.
  *   - The device error word lives in that array and cannot be read back;
  *     out-of-range lengths are still clamped exactly as in saga_decode_step.
+ *     A step kernel that gives up a bounded wait (the error that
+ *     saga_decode_step would report as SAGA_DEVERR_TIMEOUT) cannot report
+ *     it here either: instead it poisons its output, every out[b][j][:] of
+ *     the call NaN and every sel_count -1, so that the caller sees the
+ *     failure in the results.
  */
-#define SAGA_NOALLOC_SCRATCH_BYTES (4u << 20)
+#define SAGA_NOALLOC_SCRATCH_BYTES (160u << 20)
 saga_status saga_decode_step_noalloc(const saga_shape *shape, const void *q,
                                      const void *K, const void *V,
                                      const int32_t *l_kv, const float *tau,

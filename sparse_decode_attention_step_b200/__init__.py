@@ -208,7 +208,7 @@ def append_kv(shp, k_new, v_new, K, V, l_kv, ws, stream=None):
                                  _ptr(l_kv), p, n, _stream(stream)), "saga_append_kv")
 
 
-NOALLOC_SCRATCH_BYTES = 4 << 20
+NOALLOC_SCRATCH_BYTES = 160 << 20
 
 
 def decode_step_noalloc(shp, q, K, V, l_kv, tau, out, sel_count=None, stream=None):

@@ -29,12 +29,12 @@ def planned_scratch_bytes(B, h_q, h_k, h_v, d, L):
     float record per (b, j, gather split); and, per (b, j) and 32-position
     block, a 4-byte kept mask and 32 4-byte kept scores. Each part is rounded
     up to 256 bytes. The gather splits each (b, j) row so that all rows take
-    at most 888 CTAs (more only when there are more rows), each at least 8
+    at most 1184 CTAs (more only when there are more rows), each at least 8
     blocks long."""
     up = lambda x: -(-x // 256) * 256
     cdiv = lambda a, b: -(-a // b)
     nblk = cdiv(L, 32)
-    sb = min(max(1, nblk // 8), max(1, 888 // (B * h_q)))
+    sb = min(max(1, nblk // 8), max(1, 1184 // (B * h_q)))
     bps = cdiv(nblk, sb)
     SB = cdiv(nblk, bps)
     lists = B * h_q * nblk
@@ -83,13 +83,13 @@ def test_noalloc_matches_workspace_step_twice():
 
 
 def test_noalloc_scratch_limit_both_sides():
-    """The largest batch of 128-position sequences (h_q=16, h_k=2, h_v=4,
-    d=64) whose scratch fits the 4 MiB array runs and matches
+    """The largest batch of 128K-position sequences (h_q=16, h_k=2, h_v=4,
+    d=64) whose scratch fits the fixed array runs and matches
     saga_decode_step; one sequence more is refused before anything runs."""
     lib = saga.load()
     limit = saga.NOALLOC_SCRATCH_BYTES
-    L, h_q, h_k, h_v, d = 128, 16, 2, 4, 64
-    under = max(B for B in range(1, 4096) if planned_scratch_bytes(B, h_q, h_k, h_v, d, L) <= limit)
+    L, h_q, h_k, h_v, d = 131072, 16, 2, 4, 64
+    under = max(B for B in range(1, 256) if planned_scratch_bytes(B, h_q, h_k, h_v, d, L) <= limit)
     over = under + 1
     assert planned_scratch_bytes(over, h_q, h_k, h_v, d, L) > limit
 
@@ -108,6 +108,7 @@ def test_noalloc_scratch_limit_both_sides():
     sdev.fill(V, w, 0, "V")
     lens = np.full(under, L, dtype=np.int32)
     lens[::7] = 77                                # ragged tails too
+    lens[1::5] = L - 45
     shp = saga.shape(under, h_q, h_k, h_v, d, synth.BF16, L)
     ch = Chain(shp, K, V, lens, w.N, dump=False)
     qs = synth.queries(w, 0, 2)
