@@ -7,16 +7,17 @@
 // online-softmax records (m, l, count, acc[d]) for each query head, the
 // records the combine kernel merges into out.
 //
-// One CTA of four warps per (b, j, split), several CTAs per SM. A warp
-// walks its share of the split's blocks, loading up to 256 blocks' masks at
-// once (one lane per block), and lists the kept positions of consecutive
-// blocks in shared memory (block, key, rank), in position order. The rows
-// are then taken kBatch at a time: each lane copies (cp.async) its 16-byte
-// chunk of a row of value head floor(j * h_v / h_q) (d/8 lanes per row), and
-// one lane per row the row's score, into the warp's staging area, so the rows in
-// flight cost no registers and every SM has several hundred of them in
-// flight, which the latency of random row reads needs. After the copies
-// land, each lane group folds its rows into one online-softmax state (every
+// One CTA of four warps per (b, j, split), eight CTAs per SM. A warp walks
+// its share of the split's blocks, loading up to 256 blocks' masks at once
+// (one lane per block), and lists the kept positions of each group of 32
+// blocks in shared memory (block, key, rank), in position order. Each listed
+// row is issued at once into the next free slot of the warp's staging area:
+// each lane copies (cp.async) its 16-byte chunk of a row of value head
+// floor(j * h_v / h_q) (d/8 lanes per row), and one lane per row the row's
+// score, so the rows in flight cost no registers and every SM has several
+// hundred of them in flight, which the latency of random row reads needs.
+// When the kBatch slots are full, the copies land and each lane group folds
+// its rows into one online-softmax state (every
 // FMA does useful work: a row kept by several heads of one value head is
 // read once per head, about 3% more rows on the workloads here); the lane
 // groups and then the warps merge in a fixed order, so the result does not
@@ -46,10 +47,9 @@ struct GCfg {
   static constexpr int kRows = 8;             // rows per lane group and batch
   static constexpr int kBatch = NG * kRows;   // rows per warp and batch: 32 (d 64), 16 (d 128)
   static constexpr int kRec = D + kRecPad;
-  // per warp: the list of kept rows (u32 entries, kListCap of them), the
-  // staged V rows and the staged scores
-  static constexpr int kListCap = 1024;
-  static constexpr int kListBytes = kListCap * 4;
+  // per warp: a 32-block group's list of kept rows (u16 entries), the staged
+  // V rows and the staged scores
+  static constexpr int kListBytes = 32 * 32 * 2;
   static constexpr int kVBytes = kBatch * D * 2;
   static constexpr int kScBytes = kBatch * 4;
   static constexpr int kWarpBytes = kListBytes + kVBytes + kScBytes;
@@ -58,7 +58,7 @@ struct GCfg {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 6) gather_kernel(const GatherParams p) {
+__global__ void __launch_bounds__(kThreads, 8) gather_kernel(const GatherParams p) {
   using C = GCfg<D>;
   constexpr int LPG = C::LPG, NG = C::NG, kRows = C::kRows, kBatch = C::kBatch;
   extern __shared__ __align__(16) uint8_t gsm[];
@@ -96,7 +96,7 @@ __global__ void __launch_bounds__(kThreads, 6) gather_kernel(const GatherParams 
   const float *sco = p.lscore + static_cast<int64_t>(bj) * p.nblk * 32;
   const uint16_t *vrow = p.V + b * p.v_sb + static_cast<int64_t>(vh) * p.v_sh;
   uint8_t *wbase = gsm + warp * C::kWarpBytes;
-  uint32_t *list = reinterpret_cast<uint32_t *>(wbase);
+  uint16_t *list = reinterpret_cast<uint16_t *>(wbase);
   uint16_t *vst = reinterpret_cast<uint16_t *>(wbase + C::kListBytes);
   float *sst = reinterpret_cast<float *>(wbase + C::kListBytes + C::kVBytes);
 
@@ -105,71 +105,80 @@ __global__ void __launch_bounds__(kThreads, 6) gather_kernel(const GatherParams 
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 
-  // Fold the listed rows [0, total) in batches of kBatch: each lane copies
-  // its chunk of a row's V and one lane per row its score, then the lane
-  // groups fold their rows (row i goes to lane group i % NG).
+  // Staging: kBatch row slots per warp; slot i belongs to lane group i % NG.
+  // Rows are issued into the next free slots as their group's list is read
+  // (each lane copies its chunk of a row's V, one lane per row the row's
+  // score); when all kBatch slots hold rows in flight, the warp waits for
+  // them and folds them. So every wait covers a full batch, and the copies
+  // of a partly filled batch stay in flight while the next groups' lists
+  // are built.
+  int nst = 0;                         // slots issued since the last fold
+  auto fold = [&](int nb) {
+    sm100::cp_async_commit();
+    sm100::cp_async_wait_all();
+    __syncwarp();
+    float mnew = m;
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) {
+      const int i = NG * r + lg;
+      if (i < nb) mnew = fmaxf(mnew, sst[i]);
+    }
+    if (mnew != m) {
+      const float corr = exp2f((m - mnew) * kLog2e);      // 0 while m = -inf
+      m = mnew;
+      l *= corr;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] *= corr;
+    }
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) {
+      if (NG * r >= nb) break;
+      const int i = NG * r + lg;
+      if (i < nb) {
+        const float pw = exp2f((sst[i] - m) * kLog2e);
+        const uint4 x = *reinterpret_cast<const uint4 *>(vst + i * D + c * 8);
+        const float vf[8] = {bf16lo(x.x), bf16hi(x.x), bf16lo(x.y), bf16hi(x.y),
+                             bf16lo(x.z), bf16hi(x.z), bf16lo(x.w), bf16hi(x.w)};
+        l += pw;
+        ++cnt;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = fmaf(pw, vf[e], acc[e]);
+      }
+    }
+    __syncwarp();            // the staged rows are read before the next copies
+  };
+  // Issue the listed rows [0, total) of the group of blocks from gb0.
   auto run_list = [&](int total, int64_t gb0) {
-    for (int base = 0; base < total; base += kBatch) {
-      const int nb = min(kBatch, total - base);
+    for (int pos = 0; pos < total;) {
+      const int n = min(kBatch - nst, total - pos);
 #pragma unroll
       for (int r = 0; r < kRows; ++r) {
         const int i = NG * r + lg;
-        if (i < nb) {
-          const uint32_t en = list[base + i];
+        if (i >= nst && i < nst + n) {
+          const uint32_t en = list[pos + i - nst];
           const int64_t blk = gb0 + (en >> 10);
           const int64_t t = blk * 32 + ((en >> 5) & 31);
           sm100::cp_async16(vst + i * D + c * 8, vrow + t * D + c * 8);
           if (c == 0) sm100::cp_async4(sst + i, sco + blk * 32 + (en & 31));
         }
       }
-      sm100::cp_async_commit();
-      sm100::cp_async_wait_all();
-      __syncwarp();
-      // fold the batch into the lane group's state
-      float mnew = m;
-#pragma unroll
-      for (int r = 0; r < kRows; ++r) {
-        const int i = NG * r + lg;
-        if (i < nb) mnew = fmaxf(mnew, sst[i]);
+      nst += n;
+      pos += n;
+      if (nst == kBatch) {
+        fold(kBatch);
+        nst = 0;
       }
-      if (mnew != m) {
-        const float corr = exp2f((m - mnew) * kLog2e);      // 0 while m = -inf
-        m = mnew;
-        l *= corr;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] *= corr;
-      }
-#pragma unroll
-      for (int r = 0; r < kRows; ++r) {
-        if (NG * r >= nb) break;
-        const int i = NG * r + lg;
-        if (i < nb) {
-          const float pw = exp2f((sst[i] - m) * kLog2e);
-          const uint4 x = *reinterpret_cast<const uint4 *>(vst + i * D + c * 8);
-          const float vf[8] = {bf16lo(x.x), bf16hi(x.x), bf16lo(x.y), bf16hi(x.y),
-                               bf16lo(x.z), bf16hi(x.z), bf16lo(x.w), bf16hi(x.w)};
-          l += pw;
-          ++cnt;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[e] = fmaf(pw, vf[e], acc[e]);
-        }
-      }
-      __syncwarp();            // the staged rows are read before the next copies
     }
   };
 
   // this warp's blocks: an even share of the split, in order, taken in
   // chunks of up to kChunkGroups groups of 32 blocks whose masks are loaded
-  // at once (one lane per block); the kept rows of consecutive groups are
-  // listed, relative to the first listed group's block gb0, as
-  // (block offset << 10 | key << 5 | rank), and the list is folded whenever
-  // the next group might not fit, so every batch but a list's last is full
+  // at once (one lane per block), so a group's list waits for no load; each
+  // group's kept rows are listed as (block lane << 10 | key << 5 | rank)
   constexpr int kChunkGroups = 8;
   const int64_t nbs = blk1 - blk0;
   const int64_t per = (nbs + kWarps - 1) / kWarps;
   const int64_t wb0 = blk0 + min(nbs, per * warp), wb1 = blk0 + min(nbs, per * (warp + 1));
-  int listed = 0;
-  int64_t gb0 = wb0;
   for (int64_t cb = wb0; cb < wb1; cb += 32 * kChunkGroups) {
     uint32_t mks[kChunkGroups];
 #pragma unroll
@@ -190,24 +199,18 @@ __global__ void __launch_bounds__(kThreads, 6) gather_kernel(const GatherParams 
         if (lane >= o) incl += y;
       }
       const int total = __shfl_sync(0xffffffffu, incl, 31);
-      // a list whose offsets would pass 10 bits, or whose space might not
-      // hold this group, is folded first
-      if (listed > 0 && (listed + total > C::kListCap || bb - gb0 > 1023 - 31)) {
-        run_list(listed, gb0);
-        listed = 0;
-      }
-      if (listed == 0) gb0 = bb;
-      const uint32_t off = static_cast<uint32_t>(bb - gb0) + lane;
-      for (int e = listed + incl - cn, rank = 0; mk != 0u; ++e, ++rank) {
+      if (total == 0) continue;
+      for (int e = incl - cn, rank = 0; mk != 0u; ++e, ++rank) {
         const int k = __ffs(mk) - 1;
         mk &= mk - 1u;
-        list[e] = (off << 10) | static_cast<uint32_t>(k << 5) | static_cast<uint32_t>(rank);
+        list[e] = static_cast<uint16_t>((lane << 10) | (k << 5) | rank);
       }
       __syncwarp();
-      listed += total;
+      run_list(total, bb);
+      __syncwarp();          // the list is read before the next group's is written
     }
   }
-  if (listed > 0) run_list(listed, gb0);
+  if (nst > 0) fold(nst);
 
   // the warp's lane groups, merged by xor shuffles (a fixed order)
   {

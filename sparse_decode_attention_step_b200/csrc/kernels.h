@@ -49,9 +49,16 @@ cudaError_t launch_combine(const float *partials, const int32_t *l_kv, int32_t *
 // tie: nullable [B][h_q]; receives the position of the last entry equal to
 // tau that the N largest take when ties go to the lower position (one more
 // pass over the row), or INT32_MAX when N >= l_kv[b].
+// gcand [B][h_q][gcap] (gcap a multiple of 4), gcount [B][h_q] and hist1
+// [B][h_q][256] (both zeroed before the call): with hist0, a collect kernel
+// first lists each row's digit-0 bucket in gcand and counts the bucket's
+// digit 1 in hist1 (about two CTAs per SM across the rows), and the select
+// resolves the other digits from those.
 cudaError_t launch_radix_select(const float *scores, int64_t row_stride, const int32_t *l_kv,
                                 int N, float *tau, int B, int h_q, int64_t cap, int64_t max_l_kv,
-                                const uint32_t *hist0, int32_t *tie, cudaStream_t st);
+                                const uint32_t *hist0, int32_t *tie, uint32_t *gcand,
+                                uint32_t *gcount, uint32_t *hist1, int gcap, int sms,
+                                cudaStream_t st);
 
 // Dense (full-attention) split kernel over grid (S, B * h_k): GQA (h_k == h_v,
 // h_q / h_k <= 16) or SAGA heads (h_v / h_k in {2, 4}, h_q / h_k in {4, 8, 12, 16}).

@@ -8,20 +8,28 @@
 // the remaining rank. After four digits the prefix is the full key of an
 // element of the row, so tau is always one of the row's own scores.
 //
-// One CTA of 512 threads per row, two CTAs per SM, launched with programmatic
-// stream serialisation after the score pass. Digit 0 comes from the histogram the score pass already
-// built (or from one pass over the row). A second pass over the row fixes
-// digit 1 and copies the keys of the digit-0 bucket into shared memory; the
-// last two digits are found there. When that bucket does not fit (its scores
-// share one binade), a third pass copies only the keys that match the first
-// two digits; only if even those do not fit, digits 2 and 3 take one pass
-// over the row each.
+// Digit 0 comes from the histogram the score pass already built (or from one
+// pass over the row). With that histogram, a collect kernel spread over the
+// whole GPU (about two CTAs per SM, each on one segment of a row) reads every
+// row once, lists the keys of its digit-0 bucket (the keys that share the
+// N-th largest's top byte: a few percent of an attention score row, up to a
+// third when the N-th largest lies just below a power of two, since the top
+// byte spans two binades) in global memory and counts their digit 1. Then
+// one CTA of 512 threads per row takes digit 1 from that count, reads the
+// list once to keep the keys of the 16-bit prefix (tens to hundreds) in
+// shared memory, and finds the last two digits there. Without the histogram
+// (or when the bucket overflows its list, half a row), a pass over the row
+// fixes digit 1 and keeps the digit-0 bucket on chip; when that does not
+// fit, a second pass keeps the 16-bit prefix's keys; only if even those do
+// not fit, digits 2 and 3 take one pass each. Both kernels are launched with
+// programmatic stream serialisation after the score pass.
 //
 // Exact top-N (Eq. 6 with ties to the lower position) also needs, when tau is
 // tied, how far along the row the taken ties reach: after the last digit the
 // rank left inside tau's bucket is the number k of entries equal to tau that
 // the N largest include, and one more pass in position order finds the
 // position of the k-th of them.
+#include <algorithm>
 #include <atomic>
 
 #include "common.cuh"
@@ -129,6 +137,20 @@ __device__ __forceinline__ void for_row(const float *row, int64_t L, int tid, F 
   });
 }
 
+// Append k to cand when `in` (as many as fit; sh.n_cand counts them all).
+// All lanes of the warp call it together.
+__device__ __forceinline__ void append(uint32_t k, bool in, int lane, Shared &sh, uint32_t *cand) {
+  const uint32_t bal = __ballot_sync(0xffffffffu, in);
+  if (bal == 0u) return;
+  uint32_t base = 0;
+  if (lane == 0) base = atomicAdd(&sh.n_cand, static_cast<uint32_t>(__popc(bal)));
+  base = __shfl_sync(0xffffffffu, base, 0);
+  if (in) {
+    const uint32_t at = base + __popc(bal & ((1u << lane) - 1u));
+    if (at < static_cast<uint32_t>(kCand)) cand[at] = k;
+  }
+}
+
 // Copy the keys of the row with (key & mask) == prefix into cand (as many as
 // fit; the returned count may exceed kCand) and, when `shift` >= 0, count
 // digit `shift` of those keys into hist. One shared atomic per warp and step
@@ -170,11 +192,97 @@ __device__ __forceinline__ void collect(const float *row, int64_t L, int tid, in
   });
 }
 
+// The digit-0 bucket of a row (the keys whose top byte is that of the N-th
+// largest, found from the score pass's histogram), collected by `segs` CTAs
+// per row, each reading one segment of the row once: the keys go to the
+// row's list in global memory (gcap of them at most; the count may exceed
+// it, and the select then reads the row itself), one global atomic per warp
+// and step reserving the warp's places, and their digit 1 is counted into
+// the row's histogram hist1 (per-warp shared bins, added to hist1 at the
+// end). The list's order depends on timing; the select uses it as a
+// multiset only.
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+radix_collect_kernel(const float *__restrict__ scores, int64_t row_stride,
+                     const int32_t *__restrict__ l_kv, int N, int h_q, int64_t cap,
+                     int64_t max_l_kv, const uint32_t *__restrict__ hist0,
+                     uint32_t *__restrict__ gcand, uint32_t *__restrict__ gcount,
+                     uint32_t *__restrict__ hist1, int gcap, int segs) {
+  __shared__ Shared sh;
+  __shared__ uint32_t h1[kWarps][256];
+  pdl_wait();
+  pdl_trigger();
+  const int bj = blockIdx.x / segs, seg = blockIdx.x % segs;
+  const int b = bj / h_q;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int64_t L = l_kv[b];
+  const int64_t hi = cap < max_l_kv ? cap : max_l_kv;
+  if (L < 0) L = 0;
+  if (L > hi) L = hi;
+  if (static_cast<int64_t>(N) >= L) return;
+  const int64_t span = (L + segs - 1) / segs;
+  const int64_t t_lo = min(L, (span + 15) / 16 * 16 * seg);
+  const int64_t t_hi = min(L, t_lo + (span + 15) / 16 * 16);
+  if (t_lo >= t_hi) return;
+  if (tid == 0) sh.rem = static_cast<uint32_t>(N);
+  for (int i = tid; i < 256; i += kThreads) sh.hist[i] = hist0[static_cast<int64_t>(bj) * 256 + i];
+  for (int i = tid; i < kWarps * 256; i += kThreads) (&h1[0][0])[i] = 0u;
+  __syncthreads();
+  if (warp == 0) pick_digit(sh, lane);
+  __syncthreads();
+  const uint32_t d0 = sh.digit;
+  const float *row = scores + static_cast<int64_t>(bj) * row_stride + t_lo;
+  const int64_t len = t_hi - t_lo;
+  uint32_t *dst = gcand + static_cast<int64_t>(bj) * gcap;
+  uint32_t *mine = h1[warp];
+  for_row_steps(row, len, tid, [&](const float (&v)[kVec][4], int64_t t0) {
+    const bool full = t0 + kStep <= len;
+    uint32_t key[kVec * 4], in = 0;
+#pragma unroll
+    for (int u = 0; u < kVec; ++u)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        key[u * 4 + e] = order_key(v[u][e]);
+        const bool valid = full || elem_index(t0, tid, u, e) < len;
+        if (valid && (key[u * 4 + e] >> 24) == d0) in |= 1u << (u * 4 + e);
+      }
+    const uint32_t c = __popc(in);
+    uint32_t incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
+    if (total == 0u) return;
+    uint32_t base = 0;
+    if (lane == 31) base = atomicAdd(gcount + bj, total);
+    uint32_t at = __shfl_sync(0xffffffffu, base, 31) + incl - c;
+#pragma unroll
+    for (int x = 0; x < kVec * 4; ++x) {
+      if ((in >> x) & 1u) {
+        if (at < static_cast<uint32_t>(gcap)) dst[at] = key[x];
+        ++at;
+        atomicAdd(&mine[(key[x] >> 16) & 0xFFu], 1u);
+      }
+    }
+  });
+  __syncthreads();
+  uint32_t *h1_row = hist1 + static_cast<int64_t>(bj) * 256;
+  for (int i = tid; i < 256; i += kThreads) {
+    uint32_t sum = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) sum += h1[w][i];
+    if (sum != 0u) atomicAdd(h1_row + i, sum);
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 radix_select_kernel(const float *__restrict__ scores, int64_t row_stride,
                     const int32_t *__restrict__ l_kv, int N, float *__restrict__ tau, int h_q,
                     int64_t cap, int64_t max_l_kv, const uint32_t *__restrict__ hist0,
-                    int32_t *__restrict__ tie) {
+                    int32_t *__restrict__ tie, const uint32_t *__restrict__ gcand,
+                    const uint32_t *__restrict__ gcount, const uint32_t *__restrict__ hist1,
+                    int gcap) {
   __shared__ Shared sh;
   extern __shared__ uint32_t cand[];
   pdl_wait();
@@ -213,31 +321,77 @@ radix_select_kernel(const float *__restrict__ scores, int64_t row_stride,
   uint32_t prefix = sh.digit << 24, mask = 0xFF000000u;
   __syncthreads();
 
-  // ---- digit 1: one pass over the row; keep the digit-0 bucket on chip -----
-  for (int i = tid; i < 256; i += kThreads) sh.hist[i] = 0u;
-  __syncthreads();
-  collect(row, L, tid, lane, mask, prefix, 16, sh, cand);
-  __syncthreads();
-  if (warp == 0) pick_digit(sh, lane);
-  __syncthreads();
-  prefix |= sh.digit << 16;
-  mask |= 0x00FF0000u;
-  uint32_t n_cand = sh.n_cand;
-  bool on_chip = n_cand <= static_cast<uint32_t>(kCand);
-  __syncthreads();
-  if (!on_chip) {
-    // the top-byte bucket was too big: collect the (much smaller) bucket of
-    // the 16-bit prefix instead, with one more pass over the row
-    if (tid == 0) sh.n_cand = 0;
+  // ---- digit 1, and the keys kept on chip ---------------------------------
+  // With the collect kernel's list of the digit-0 bucket (when it fit) and
+  // its digit-1 histogram, digit 1 needs no pass; the list is read once to
+  // keep the keys of the 16-bit prefix on chip. Otherwise one pass over the
+  // row fixes digit 1 and keeps the digit-0 bucket on chip.
+  const uint32_t n_g = gcand != nullptr ? gcount[bj] : 0xFFFFFFFFu;
+  const bool listed = n_g <= static_cast<uint32_t>(gcap);
+  const uint32_t *list = listed ? gcand + static_cast<int64_t>(bj) * gcap : nullptr;
+  // visit the list (16-byte loads, kVec per thread in flight) or the row
+  auto for_src = [&](auto f) {
+    if (listed) {
+      const uint4 *l4 = reinterpret_cast<const uint4 *>(list);
+      const uint32_t n4 = (n_g + 3u) / 4u;            // within gcap (a multiple of 4)
+      for (uint32_t i0 = 0; i0 < n4; i0 += kThreads * kVec) {
+        uint4 x[kVec];
+#pragma unroll
+        for (int u = 0; u < kVec; ++u) {
+          const uint32_t i = i0 + u * kThreads + tid;
+          x[u] = i < n4 ? __ldcg(l4 + i) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < kVec; ++u) {
+          const uint32_t i = (i0 + u * kThreads + tid) * 4u;
+          f(x[u].x, i < n_g);
+          f(x[u].y, i + 1u < n_g);
+          f(x[u].z, i + 2u < n_g);
+          f(x[u].w, i + 3u < n_g);
+        }
+      }
+    } else {
+      for_row(row, L, tid, f);
+    }
+  };
+  uint32_t n_cand;
+  if (listed) {
+    for (int i = tid; i < 256; i += kThreads) sh.hist[i] = hist1[static_cast<int64_t>(bj) * 256 + i];
     __syncthreads();
-    collect(row, L, tid, lane, mask, prefix, -1, sh, cand);
+    if (warp == 0) pick_digit(sh, lane);
+    __syncthreads();
+    prefix |= sh.digit << 16;
+    mask |= 0x00FF0000u;
+    for_src([&](uint32_t k, bool valid) {
+      append(k, valid && (k & mask) == prefix, lane, sh, cand);
+    });
     __syncthreads();
     n_cand = sh.n_cand;
-    on_chip = n_cand <= static_cast<uint32_t>(kCand);
+  } else {
+    for (int i = tid; i < 256; i += kThreads) sh.hist[i] = 0u;
     __syncthreads();
+    collect(row, L, tid, lane, mask, prefix, 16, sh, cand);
+    __syncthreads();
+    if (warp == 0) pick_digit(sh, lane);
+    __syncthreads();
+    prefix |= sh.digit << 16;
+    mask |= 0x00FF0000u;
+    n_cand = sh.n_cand;
+    __syncthreads();
+    if (n_cand > static_cast<uint32_t>(kCand)) {
+      // the top-byte bucket was too big: keep the (much smaller) bucket of
+      // the 16-bit prefix instead, with one more pass over the row
+      if (tid == 0) sh.n_cand = 0;
+      __syncthreads();
+      collect(row, L, tid, lane, mask, prefix, -1, sh, cand);
+      __syncthreads();
+      n_cand = sh.n_cand;
+    }
   }
+  const bool on_chip = n_cand <= static_cast<uint32_t>(kCand);
+  __syncthreads();
 
-  // ---- digits 2 and 3: over the candidates, else over the row -------------
+  // ---- digits 2 and 3: over the keys on chip, else over the list or row ---
   for (int shift = 8; shift >= 0; shift -= 8) {
     for (int i = tid; i < 256; i += kThreads) sh.hist[i] = 0u;
     __syncthreads();
@@ -248,7 +402,7 @@ radix_select_kernel(const float *__restrict__ scores, int64_t row_stride,
         count_key(k, i < n_cand, mask, prefix, shift, sh.hist, lane);
       }
     } else {
-      for_row(row, L, tid, [&](uint32_t k, bool valid) {
+      for_src([&](uint32_t k, bool valid) {
         count_key(k, valid, mask, prefix, shift, sh.hist, lane);
       });
     }
@@ -311,7 +465,9 @@ radix_select_kernel(const float *__restrict__ scores, int64_t row_stride,
 
 cudaError_t launch_radix_select(const float *scores, int64_t row_stride, const int32_t *l_kv,
                                 int N, float *tau, int B, int h_q, int64_t cap, int64_t max_l_kv,
-                                const uint32_t *hist0, int32_t *tie, cudaStream_t st) {
+                                const uint32_t *hist0, int32_t *tie, uint32_t *gcand,
+                                uint32_t *gcount, uint32_t *hist1, int gcap, int sms,
+                                cudaStream_t st) {
   // the dynamic shared-memory opt-in is per device; set once on each
   static std::atomic<bool> attr_set[kMaxDevices];
   const int smem = kCand * static_cast<int>(sizeof(uint32_t));
@@ -325,8 +481,23 @@ cudaError_t launch_radix_select(const float *scores, int64_t row_stride, const i
     if (e != cudaSuccess) return e;
     attr_set[dev].store(true, std::memory_order_release);
   }
-  return launch_pdl(radix_select_kernel, dim3(B * h_q), dim3(kThreads), smem, st, scores,
-                    row_stride, l_kv, N, tau, h_q, cap, max_l_kv, hist0, tie);
+  const int rows = B * h_q;
+  const bool two_pass = hist0 != nullptr && gcand != nullptr && gcount != nullptr &&
+                        hist1 != nullptr && gcap > 0 && gcap % 4 == 0;
+  if (two_pass) {
+    // enough segments per row to give every SM two CTAs, each at least 16K positions long
+    const int64_t by_sms = std::max<int64_t>(1, static_cast<int64_t>(kCtasPerSm) * sms / rows);
+    const int64_t by_len = std::max<int64_t>(1, max_l_kv / 16384);
+    const int segs = static_cast<int>(std::min(by_sms, by_len));
+    e = launch_pdl(radix_collect_kernel, dim3(rows * segs), dim3(kThreads), 0, st, scores,
+                   row_stride, l_kv, N, h_q, cap, max_l_kv, hist0, gcand, gcount, hist1, gcap,
+                   segs);
+    if (e != cudaSuccess) return e;
+  }
+  return launch_pdl(radix_select_kernel, dim3(rows), dim3(kThreads), smem, st, scores,
+                    row_stride, l_kv, N, tau, h_q, cap, max_l_kv, hist0, tie,
+                    two_pass ? gcand : nullptr, two_pass ? gcount : nullptr,
+                    two_pass ? hist1 : nullptr, gcap);
 }
 
 }  // namespace saga

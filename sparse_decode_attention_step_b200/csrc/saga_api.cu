@@ -34,8 +34,19 @@ struct Plan {
   // the records the combine merges: comb_S per (b, j), comb_split_len positions each
   int comb_S;
   int64_t comb_split_len;
-  size_t off_partials, off_lmask, off_lscore, off_scores, off_hist, off_tau, off_tie, total;
+  // radix select: per row, the list of the top-byte bucket (gcap keys at most)
+  int gcap;
+  size_t off_partials, off_lmask, off_lscore, off_scores, off_hist, off_gcount, off_hist1,
+      off_gcand, off_tau, off_tie, total;
 };
+
+// Keys per row in the radix select's bucket list: half the row (the top-byte
+// bucket of a score row can hold a third of it), at least 16384, a multiple
+// of 4.
+int select_list_cap(int64_t max_l_kv) {
+  const int64_t c = std::max<int64_t>(16384, (max_l_kv / 2 + 3) / 4 * 4);
+  return static_cast<int>(c);
+}
 
 bool use_tc(const saga_shape &s);
 
@@ -48,10 +59,10 @@ bool use_tc(const saga_shape &s);
 // more splits than slots only add waves and combine work.
 // Persistent tensor-core scan: at most one unit per SM and wave, units of up
 // to about kPersistTiles tiles. Its gather kernel splits each (b, query head)
-// row on its own, into at most kGatherCtas CTAs in all (one wave, six
+// row on its own, into at most kGatherCtas CTAs in all (one wave, eight
 // resident per SM) where the rows allow, each at least kGatherMinBlocks
 // blocks of 32 positions long; the combine merges the gather's records.
-constexpr int64_t kGatherCtas = 6 * kSms;
+constexpr int64_t kGatherCtas = 8 * kSms;
 constexpr int64_t kGatherMinBlocks = 8;
 
 Plan make_plan(const saga_shape &s, bool persistent, int64_t ctas_per_sm = kGridCtasPerSm) {
@@ -90,7 +101,13 @@ Plan make_plan(const saga_shape &s, bool persistent, int64_t ctas_per_sm = kGrid
   p.off_lscore = align_up(p.off_lmask + lists * sizeof(uint32_t));
   p.off_scores = align_up(p.off_lscore + lists * 32 * sizeof(float));
   p.off_hist = align_up(p.off_scores + static_cast<size_t>(s.B) * s.h_q * s.max_l_kv * sizeof(float));
-  p.off_tau = align_up(p.off_hist + static_cast<size_t>(s.B) * s.h_q * 256 * sizeof(uint32_t));
+  // the bucket counts and digit-1 histograms follow the top-byte histograms
+  // directly: one memset clears all three
+  p.gcap = select_list_cap(s.max_l_kv);
+  p.off_gcount = p.off_hist + static_cast<size_t>(s.B) * s.h_q * 256 * sizeof(uint32_t);
+  p.off_hist1 = p.off_gcount + static_cast<size_t>(s.B) * s.h_q * sizeof(uint32_t);
+  p.off_gcand = align_up(p.off_hist1 + static_cast<size_t>(s.B) * s.h_q * 256 * sizeof(uint32_t));
+  p.off_tau = align_up(p.off_gcand + static_cast<size_t>(s.B) * s.h_q * p.gcap * sizeof(uint32_t));
   p.off_tie = align_up(p.off_tau + static_cast<size_t>(s.B) * s.h_q * sizeof(float));
   p.total = align_up(p.off_tie + static_cast<size_t>(s.B) * s.h_q * sizeof(int32_t));
   return p;
@@ -228,6 +245,23 @@ saga_status run_dense(const saga_shape &s, const void *q, const void *K, const v
 
 thread_local char g_last_error[256] = "";
 
+// The top-byte histograms the score pass fills, and the bucket counts and
+// digit-1 histograms of the radix select, cleared together (they are
+// adjacent in the workspace).
+struct SelectBufs {
+  uint32_t *hist = nullptr, *gcount = nullptr, *hist1 = nullptr, *gcand = nullptr;
+};
+cudaError_t clear_select_counts(const saga_shape &s, const Plan &pl, void *ws, SelectBufs *b,
+                                cudaStream_t st) {
+  char *wsb = static_cast<char *>(ws);
+  b->hist = reinterpret_cast<uint32_t *>(wsb + pl.off_hist);
+  b->gcount = reinterpret_cast<uint32_t *>(wsb + pl.off_gcount);
+  b->hist1 = reinterpret_cast<uint32_t *>(wsb + pl.off_hist1);
+  b->gcand = reinterpret_cast<uint32_t *>(wsb + pl.off_gcand);
+  const size_t rows = static_cast<size_t>(s.B) * s.h_q;
+  return cudaMemsetAsync(b->hist, 0, rows * (256 + 1 + 256) * sizeof(uint32_t), st);
+}
+
 }  // namespace
 
 saga_status cuda_fail(cudaError_t e, const char *where) {
@@ -331,20 +365,20 @@ saga_status saga_refresh_threshold(const saga_shape *shape, const void *q, const
                     ? scores
                     : reinterpret_cast<float *>(static_cast<char *>(ws) + pl.off_scores);
   // 1. score rows (tensor-core kernel: with the top-byte histogram of every row)
-  uint32_t *hist = nullptr;
+  SelectBufs sb;
   if (use_tc(s)) {
-    hist = reinterpret_cast<uint32_t *>(static_cast<char *>(ws) + pl.off_hist);
-    const cudaError_t me =
-        cudaMemsetAsync(hist, 0, static_cast<size_t>(s.B) * s.h_q * 256 * sizeof(uint32_t), st);
+    const cudaError_t me = clear_select_counts(s, pl, ws, &sb, st);
     if (me != cudaSuccess) return cuda_fail(me, "cudaMemsetAsync (histograms)");
   }
+  uint32_t *hist = sb.hist;
   p.scores_out = rows;
   p.hist = hist;
   cudaError_t e = launch_split(s, p, kModeDump, st);
   if (e != cudaSuccess) return cuda_fail(e, "score dump kernel");
   // 2. exact N-th largest per row
   e = launch_radix_select(rows, s.max_l_kv, l_kv, N, tau, s.B, s.h_q, s.cap, s.max_l_kv, hist,
-                          nullptr, st);
+                          nullptr, sb.gcand, sb.gcount, sb.hist1, pl.gcap, static_cast<int>(kSms),
+                          st);
   if (e != cudaSuccess) return cuda_fail(e, "radix select kernel");
   if (V == nullptr) return SAGA_OK;
   // 3. this step's select + PV with the fresh tau, over the very rows tau
@@ -385,20 +419,20 @@ saga_status saga_topn_step(const saga_shape *shape, const void *q, const void *K
   float *tau = reinterpret_cast<float *>(wsb + pl.off_tau);
   int32_t *tie = reinterpret_cast<int32_t *>(wsb + pl.off_tie);
   // 1. score rows (tensor-core kernel: with the top-byte histogram of every row)
-  uint32_t *hist = nullptr;
+  SelectBufs sb;
   if (use_tc(s)) {
-    hist = reinterpret_cast<uint32_t *>(wsb + pl.off_hist);
-    const cudaError_t me =
-        cudaMemsetAsync(hist, 0, static_cast<size_t>(s.B) * s.h_q * 256 * sizeof(uint32_t), st);
+    const cudaError_t me = clear_select_counts(s, pl, ws, &sb, st);
     if (me != cudaSuccess) return cuda_fail(me, "cudaMemsetAsync (histograms)");
   }
+  uint32_t *hist = sb.hist;
   p.scores_out = rows;
   p.hist = hist;
   cudaError_t e = launch_split(s, p, kModeDump, st);
   if (e != cudaSuccess) return cuda_fail(e, "score dump kernel");
   // 2. the N-th largest and, when it is tied, the last tied position taken
   e = launch_radix_select(rows, s.max_l_kv, l_kv, N, tau, s.B, s.h_q, s.cap, s.max_l_kv, hist,
-                          tie, st);
+                          tie, sb.gcand, sb.gcount, sb.hist1, pl.gcap, static_cast<int>(kSms),
+                          st);
   if (e != cudaSuccess) return cuda_fail(e, "radix select kernel");
   // 3. the step over exactly those positions, from the stored rows (or, on
   // the tensor-core path when they cannot be streamed, from bit-identical
