@@ -230,15 +230,15 @@ saga_status saga_append_kv(const saga_shape *shape, const void *k_new,
  *   - On the tensor-core path the step needs, each part rounded up to 256
  *     bytes: 256 bytes of error and abort words; 4*B*h_q*SB*(d+4) bytes of
  *     per-split softmax states, SB being the gather splits of a (b, query
- *     head) row the library plans (at most max_l_kv/256, and no more than
- *     1184/(B*h_q) when that is larger than one); and 132*B*h_q*nblk bytes of
+ *     head) row the library plans (at most max_l_kv/2048, and no more than
+ *     4736/(B*h_q) when that is larger than one); and 132*B*h_q*nblk bytes of
  *     per-head kept lists, nblk = ceil(max_l_kv/32) (a 32-bit mask and 32
  *     fp32 kept scores per 32-position block). A shape needing more than
  *     SAGA_NOALLOC_SCRATCH_BYTES is rejected with SAGA_ERR_WORKSPACE, an
  *     invalid one with SAGA_ERR_INVALID_ARG, and nothing is enqueued then.
  *     (The 16-layer batch-8 128K Llama-3.2-1B workload, h_q = 32, needs
- *     about 139 MB per layer call; batch-1 128K Qwen2.5-1.5B, h_q = 12,
- *     about 7.1 MB.)
+ *     about 140 MB per layer call; batch-1 128K Qwen2.5-1.5B, h_q = 12,
+ *     about 6.9 MB.)
  *   - It calls no cudaMalloc, cudaFree or other allocating routine.
  *   - The first call on each device looks up the array's device address
  *     with that device current; make that first call before any stream

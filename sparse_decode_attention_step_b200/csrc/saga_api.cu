@@ -59,11 +59,13 @@ bool use_tc(const saga_shape &s);
 // more splits than slots only add waves and combine work.
 // Persistent tensor-core scan: at most one unit per SM and wave, units of up
 // to about kPersistTiles tiles. Its gather kernel splits each (b, query head)
-// row on its own, into at most kGatherCtas CTAs in all (one wave, eight
-// resident per SM) where the rows allow, each at least kGatherMinBlocks
-// blocks of 32 positions long; the combine merges the gather's records.
-constexpr int64_t kGatherCtas = 8 * kSms;
-constexpr int64_t kGatherMinBlocks = 8;
+// row on its own, into at most kGatherCtas CTAs in all (about four waves of
+// eight resident per SM, so that heads that keep more rows than others are
+// balanced out by the block scheduler) where the rows allow, each at least
+// kGatherMinBlocks blocks of 32 positions long; the combine merges the
+// gather's records.
+constexpr int64_t kGatherCtas = 32 * kSms;
+constexpr int64_t kGatherMinBlocks = 64;
 
 Plan make_plan(const saga_shape &s, bool persistent, int64_t ctas_per_sm = kGridCtasPerSm) {
   Plan p{};

@@ -29,12 +29,12 @@ def planned_scratch_bytes(B, h_q, h_k, h_v, d, L):
     float record per (b, j, gather split); and, per (b, j) and 32-position
     block, a 4-byte kept mask and 32 4-byte kept scores. Each part is rounded
     up to 256 bytes. The gather splits each (b, j) row so that all rows take
-    at most 1184 CTAs (more only when there are more rows), each at least 8
+    at most 4736 CTAs (more only when there are more rows), each at least 64
     blocks long."""
     up = lambda x: -(-x // 256) * 256
     cdiv = lambda a, b: -(-a // b)
     nblk = cdiv(L, 32)
-    sb = min(max(1, nblk // 8), max(1, 1184 // (B * h_q)))
+    sb = min(max(1, nblk // 64), max(1, 4736 // (B * h_q)))
     bps = cdiv(nblk, sb)
     SB = cdiv(nblk, bps)
     lists = B * h_q * nblk
