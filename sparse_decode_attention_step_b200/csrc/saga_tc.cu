@@ -204,7 +204,7 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
   const int G = p.h_q / p.h_k;
   const int n_units = p.B * p.h_k * p.S;
 
-  // ---- set-up (touches no global memory) ---------------------------------
+  // ---- set-up ----------------------------------------------------------------
   if (tid == 0) {
     for (int i = 0; i < C::kStages; ++i) {
       sm100::mbar_init(&h->full[i], 1);
@@ -228,6 +228,20 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
   if (kDump && p.hist != nullptr && warp >= 2) {
     uint32_t *hs = reinterpret_cast<uint32_t *>(scratch);
     for (int i = tid - 64; i < kN * 256; i += C::kWorkers * 32) hs[i] = 0u;
+  }
+  // While the previous launch in the stream finishes, bring the first K
+  // tiles of this CTA's first unit into L2. K itself may still be written by
+  // that launch (a KV append); L2 holds the one copy every SM reads, so a
+  // line fetched early is updated by such a write, never stale.
+  if (!kDump && !FS && warp == 0 && lane == 0 && static_cast<int>(blockIdx.x) < n_units) {
+    const int u = blockIdx.x;
+    const int bk = u % (p.B * p.h_k);
+    const int64_t t0 = static_cast<int64_t>(u / (p.B * p.h_k)) * p.split_len;
+    const int n = static_cast<int>(min(static_cast<int64_t>(C::kStages), p.split_len / kTileKeys));
+    for (int i = 0; i < n; ++i)
+      for (int bx = 0; bx < C::kBoxes; ++bx)
+        sm100::tma_prefetch_4d(&kmap, bx * 64, static_cast<int>(t0) + i * kTileKeys, bk % p.h_k,
+                               bk / p.h_k);
   }
   sm100::tc_fence_before();
   __syncthreads();
