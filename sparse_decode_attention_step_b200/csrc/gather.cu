@@ -149,6 +149,9 @@ __global__ void __launch_bounds__(kThreads, 8) gather_kernel(const GatherParams 
   };
   // Issue the listed rows [0, total) of the group of blocks from gb0.
   auto run_list = [&](int total, int64_t gb0) {
+    // the group's V rows and kept scores, addressed from its first block
+    const uint16_t *vg = vrow + gb0 * 32 * D + c * 8;
+    const float *sg = sco + gb0 * 32;
     for (int pos = 0; pos < total;) {
       const int n = min(kBatch - nst, total - pos);
 #pragma unroll
@@ -156,10 +159,9 @@ __global__ void __launch_bounds__(kThreads, 8) gather_kernel(const GatherParams 
         const int i = NG * r + lg;
         if (i >= nst && i < nst + n) {
           const uint32_t en = list[pos + i - nst];
-          const int64_t blk = gb0 + (en >> 10);
-          const int64_t t = blk * 32 + ((en >> 5) & 31);
-          sm100::cp_async16(vst + i * D + c * 8, vrow + t * D + c * 8);
-          if (c == 0) sm100::cp_async4(sst + i, sco + blk * 32 + (en & 31));
+          const uint32_t bl = en >> 10;                        // block within the group
+          sm100::cp_async16(vst + i * D + c * 8, vg + (bl * 32 + ((en >> 5) & 31)) * D);
+          if (c == 0) sm100::cp_async4(sst + i, sg + bl * 32 + (en & 31));
         }
       }
       nst += n;

@@ -58,13 +58,16 @@ constexpr int kN = 16;                      // MMA N: query heads of a group, pa
 constexpr int kWorkerBar = 1;               // named barrier of the worker warps
 constexpr uint32_t kIdesc = sm100::idesc_bf16_f32(kTileKeys, kN);
 
-template <int D>
+// R: worker warps per lane quarter. The plain step's workers keep up with
+// the MMA at 3 (d = 64) and 2 (d = 128); the dump and the steps from stored
+// scores do more per tile and take 5 and 3.
+template <int D, int R>
 struct Cfg {
-  static constexpr int kRanks = D == 64 ? 3 : 2;              // worker warps per lane quarter
+  static constexpr int kRanks = R;
   static constexpr int kWorkers = 4 * kRanks;
   static constexpr int kThreads = 32 * (2 + kWorkers);
   static constexpr int kStages = D == 64 ? 8 : 4;             // 128 KB of K in flight
-  static constexpr int kTBufs = 2 * kRanks;                    // TMEM score buffers
+  static constexpr int kTBufs = 2 * kRanks <= 8 ? 2 * kRanks : 8;   // TMEM score buffers
   static constexpr int kTmemCols = kTBufs * kN <= 32 ? 32 : (kTBufs * kN <= 64 ? 64 : 128);
   static_assert(kTBufs * kN <= kTmemCols, "TMEM buffers fit the allocation");
   static constexpr int kBoxes = D / 64;                        // 64-column TMA boxes per tile
@@ -78,10 +81,10 @@ struct Cfg {
   static constexpr int kScratchBytes = kHistBytes;
 };
 
-template <int D>
+template <typename C>
 struct Header {
-  uint64_t full[Cfg<D>::kStages], empty[Cfg<D>::kStages];
-  uint64_t tfull[Cfg<D>::kTBufs], tempty[Cfg<D>::kTBufs];
+  uint64_t full[C::kStages], empty[C::kStages];
+  uint64_t tfull[C::kTBufs], tempty[C::kTBufs];
   uint64_t qfull[2], qempty[2];
   uint32_t tmem_base;
   int abort;
@@ -89,14 +92,13 @@ struct Header {
   int32_t tie[kN];           // tie mode: last position at which A == tau is kept
 };
 
-template <int D>
+template <typename C>
 struct Layout {
-  using C = Cfg<D>;
   static constexpr int off_stage = 0;
   static constexpr int off_q = C::kStages * C::kTileBytes;
   static constexpr int off_scratch = off_q + 2 * C::kQBytes;
   static constexpr int off_hdr = off_scratch + C::kScratchBytes;
-  static constexpr int bytes = off_hdr + static_cast<int>(sizeof(Header<D>));
+  static constexpr int bytes = off_hdr + static_cast<int>(sizeof(Header<C>));
   static constexpr int alloc = bytes + 1024;                  // slack for 1024-byte alignment
   static_assert(alloc <= 227 * 1024, "shared memory of one CTA");
   static_assert(off_hdr % 16 == 0 && off_q % 1024 == 0, "operand alignment");
@@ -129,13 +131,13 @@ __device__ __forceinline__ bool unit_at(const StepParams &p, int u, bool report,
   return true;
 }
 
-template <int D>
-__device__ __forceinline__ bool aborted(Header<D> *h) {
+template <typename C>
+__device__ __forceinline__ bool aborted(Header<C> *h) {
   return *reinterpret_cast<volatile int *>(&h->abort) != 0;
 }
 
-template <int D>
-__device__ __forceinline__ void fail(const StepParams &p, Header<D> *h) {
+template <typename C>
+__device__ __forceinline__ void fail(const StepParams &p, Header<C> *h) {
   if (!aborted(h)) {
     atomicOr(p.err, SAGA_DEVERR_TIMEOUT);
     if (p.abort != nullptr) atomicExch(p.abort, 1);   // the gather poisons this step's records
@@ -144,8 +146,8 @@ __device__ __forceinline__ void fail(const StepParams &p, Header<D> *h) {
 }
 
 // Bounded wait that also gives up as soon as another role has aborted.
-template <int D>
-__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Header<D> *h) {
+template <typename C>
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Header<C> *h) {
   if (sm100::mbar_test_wait(bar, parity)) return true;
   const uint64_t t0 = sm100::global_ns();
   for (;;) {
@@ -156,15 +158,15 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Header<
 }
 
 // Warp-uniform version: lane 0 waits, the verdict is broadcast.
-template <int D>
-__device__ __forceinline__ bool warp_wait_bar(uint64_t *bar, uint32_t parity, Header<D> *h) {
+template <typename C>
+__device__ __forceinline__ bool warp_wait_bar(uint64_t *bar, uint32_t parity, Header<C> *h) {
   bool ok = true;
   if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, h);
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
 // OR of `pred` over the worker warps (a barrier among them).
-template <int D>
+template <typename C>
 __device__ __forceinline__ bool workers_any(bool pred) {
   uint32_t r;
   asm volatile(
@@ -173,22 +175,25 @@ __device__ __forceinline__ bool workers_any(bool pred) {
       "bar.red.or.pred p, %2, %3, q;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(r)
-      : "r"(static_cast<uint32_t>(pred)), "r"(kWorkerBar), "r"(Cfg<D>::kWorkers * 32)
+      : "r"(static_cast<uint32_t>(pred)), "r"(kWorkerBar), "r"(C::kWorkers * 32)
       : "memory");
   return r != 0;
 }
 
-template <int D>
+template <typename C>
 __device__ __forceinline__ void workers_sync() {
-  sm100::named_bar(kWorkerBar, Cfg<D>::kWorkers * 32);
+  sm100::named_bar(kWorkerBar, C::kWorkers * 32);
 }
 
 template <int D, int MODE, bool FS>
-__global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
+using CfgOf = Cfg<D, (MODE == kModeStep && !FS) ? (D == 64 ? 3 : 2) : (D == 64 ? 5 : 3)>;
+
+template <int D, int MODE, bool FS>
+__global__ void __launch_bounds__(CfgOf<D, MODE, FS>::kThreads, 1)
 saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
                const __grid_constant__ CUtensorMap qmap) {
-  using C = Cfg<D>;
-  using Lo = Layout<D>;
+  using C = CfgOf<D, MODE, FS>;
+  using Lo = Layout<C>;
   constexpr bool kDump = MODE == kModeDump;
   static_assert(!(kDump && FS), "the dump reads K");
 
@@ -198,7 +203,7 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
   uint8_t *stages = smem + Lo::off_stage;
   uint8_t *qbuf = smem + Lo::off_q;
   float *scratch = reinterpret_cast<float *>(smem + Lo::off_scratch);
-  Header<D> *h = reinterpret_cast<Header<D> *>(smem + Lo::off_hdr);
+  Header<C> *h = reinterpret_cast<Header<C> *>(smem + Lo::off_hdr);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = p.h_q / p.h_k;
@@ -368,7 +373,7 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
           h->tau[lane] = lane < G ? p.tau[un.b * p.h_q + j0 + lane] : INFINITY;
           if (MODE == kModeStepTies) h->tie[lane] = lane < G ? p.tie[un.b * p.h_q + j0 + lane] : -1;
         }
-        workers_sync<D>();
+        workers_sync<C>();
       }
 
       const int first = (rank - static_cast<int>(g % C::kRanks) + C::kRanks) % C::kRanks;
@@ -480,7 +485,7 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
       g += un.n_tiles;
 
       // ---- end of unit -------------------------------------------------------
-      if (workers_any<D>(bad || aborted(h))) break;
+      if (workers_any<C>(bad || aborted(h))) break;
       if (kDump && p.hist != nullptr) {
         uint32_t *hs = reinterpret_cast<uint32_t *>(scratch);
         for (int i = widx * 32 + lane; i < kN * 256; i += C::kWorkers * 32) {
@@ -489,7 +494,7 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
             atomicAdd(&p.hist[static_cast<int64_t>(un.b * p.h_q + j0 + i / 256) * 256 + (i % 256)], c);
           hs[i] = 0u;
         }
-        workers_sync<D>();
+        workers_sync<C>();
       }
     }
   }
@@ -541,7 +546,7 @@ int sm_count(int dev) {
 template <int D, int MODE, bool FS>
 cudaError_t launch_tc(const StepParams &p, const CUtensorMap &kmap, const CUtensorMap &qmap,
                       int dev, cudaStream_t st) {
-  using Lo = Layout<D>;
+  using Lo = Layout<CfgOf<D, MODE, FS>>;
   static std::atomic<bool> attr_set[kMaxDevices];
   if (!attr_set[dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(saga_tc_kernel<D, MODE, FS>,
@@ -554,7 +559,7 @@ cudaError_t launch_tc(const StepParams &p, const CUtensorMap &kmap, const CUtens
   const int n_units = p.B * p.h_k * p.S;
   const int grid = n_units < sms ? n_units : sms;
   if (grid < 1) return cudaSuccess;
-  return launch_pdl(saga_tc_kernel<D, MODE, FS>, dim3(grid), dim3(Cfg<D>::kThreads), Lo::alloc,
+  return launch_pdl(saga_tc_kernel<D, MODE, FS>, dim3(grid), dim3(CfgOf<D, MODE, FS>::kThreads), Lo::alloc,
                     st, p, kmap, qmap);
 }
 
