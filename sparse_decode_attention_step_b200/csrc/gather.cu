@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(kThreads, 8) gather_kernel(const GatherParams 
   const int sb = blockIdx.x % p.SB;
   const int bj = blockIdx.x / p.SB;                  // b * h_q + j
   const int b = bj / p.h_q, j = bj % p.h_q;
-  const int vh = j / (p.h_q / p.h_v);
+  const int vh = j / p.hpv;
 
   int64_t L = p.l_kv[b];
   const int64_t hi = p.cap < p.max_l_kv ? p.cap : p.max_l_kv;
@@ -154,10 +154,12 @@ __global__ void __launch_bounds__(kThreads, 8) gather_kernel(const GatherParams 
     const float *sg = sco + gb0 * 32;
     for (int pos = 0; pos < total;) {
       const int n = min(kBatch - nst, total - pos);
-#pragma unroll
-      for (int r = 0; r < kRows; ++r) {
+      // this lane group's slots i = NG * r + lg in [nst, nst + n)
+      const int r_lo = max(0, (nst - lg + NG - 1) / NG);
+      const int r_hi = min(kRows, (nst + n - lg + NG - 1) / NG);
+      for (int r = r_lo; r < r_hi; ++r) {
         const int i = NG * r + lg;
-        if (i >= nst && i < nst + n) {
+        {
           const uint32_t en = list[pos + i - nst];
           const uint32_t bl = en >> 10;                        // block within the group
           sm100::cp_async16(vst + i * D + c * 8, vg + (bl * 32 + ((en >> 5) & 31)) * D);
