@@ -57,6 +57,14 @@ struct GCfg {
   static constexpr int kSmem = kWarps * kWarpBytes > kMergeBytes ? kWarps * kWarpBytes : kMergeBytes;
 };
 
+// 2^x by the hardware's approximate exponential (relative error near 2^-22,
+// well inside the step's tolerance); x <= 0 here, and 2^-inf = 0.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 8) gather_kernel(const GatherParams p) {
   using C = GCfg<D>;
@@ -130,17 +138,17 @@ __global__ void __launch_bounds__(kThreads, 8) gather_kernel(const GatherParams 
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[e] *= corr;
     }
+    cnt += max(0, min(kRows, (nb - lg + NG - 1) / NG));   // rows of this lane group
 #pragma unroll
     for (int r = 0; r < kRows; ++r) {
       if (NG * r >= nb) break;
       const int i = NG * r + lg;
       if (i < nb) {
-        const float pw = exp2f((sst[i] - m) * kLog2e);
+        const float pw = ex2((sst[i] - m) * kLog2e);
         const uint4 x = *reinterpret_cast<const uint4 *>(vst + i * D + c * 8);
         const float vf[8] = {bf16lo(x.x), bf16hi(x.x), bf16lo(x.y), bf16hi(x.y),
                              bf16lo(x.z), bf16hi(x.z), bf16lo(x.w), bf16hi(x.w)};
         l += pw;
-        ++cnt;
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = fmaf(pw, vf[e], acc[e]);
       }
