@@ -73,6 +73,8 @@ typedef enum saga_dtype {
 #define SAGA_DEVERR_LKV_NEGATIVE 1   /* some l_kv[b] < 0, treated as 0 */
 #define SAGA_DEVERR_LKV_TOO_LONG 2   /* some l_kv[b] > min(cap, max_l_kv), clamped */
 #define SAGA_DEVERR_TIMEOUT 4        /* a bounded on-chip wait gave up; outputs invalid */
+#define SAGA_DEVERR_BOUNDS 8         /* bounds-checked build only: an index check failed and
+                                        the access was skipped; outputs invalid */
 
 /*
  * Problem shape. Layouts (element strides, d contiguous within a row):

@@ -11,7 +11,9 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "_lib", "libsaga_b200.so")
+# SAGA_CHECKED_BUILD=1 selects the bounds-checked build (build.py --check)
+LIB_PATH = os.path.join(_HERE, "_lib", "libsaga_b200_check.so"
+                        if os.environ.get("SAGA_CHECKED_BUILD") == "1" else "libsaga_b200.so")
 
 SAGA_OK = 0
 SAGA_ERR_INVALID_ARG = 1

@@ -38,6 +38,20 @@ struct StepParams {
   float scale;              // 1 / sqrt(d)
 };
 
+// Index checks of the bounds-checked build (-DSAGA_CHECK): a failed check
+// sets SAGA_DEVERR_BOUNDS in the error word and the caller skips the access.
+// In the ordinary build every check is true at compile time.
+__device__ __forceinline__ bool saga_in_bounds(bool ok, int32_t *err) {
+#ifdef SAGA_CHECK
+  if (!ok && err != nullptr) atomicOr(err, SAGA_DEVERR_BOUNDS);
+  return ok;
+#else
+  (void)ok;
+  (void)err;
+  return true;
+#endif
+}
+
 // Clamp a device-side sequence length into [0, min(cap, max_l_kv)] and
 // record any violation in the error word.
 // Gather kernel parameters: the kept lists of a tensor-core scan, the V
@@ -52,6 +66,7 @@ struct GatherParams {
   int64_t nblk;
   float *partials;          // [B][h_q][SB][d + kRecPad]
   const int32_t *abort;     // the scan's abort word
+  int32_t *err;             // device error word (index checks of the checked build)
   int32_t B, h_q, h_v, SB;
   int32_t hpv;              // h_q / h_v: query heads per value head
   int64_t blk_per_split;    // 32-position blocks per split

@@ -170,8 +170,11 @@ __global__ void __launch_bounds__(kThreads, 8) gather_kernel(const GatherParams 
         {
           const uint32_t en = list[pos + i - nst];
           const uint32_t bl = en >> 10;                        // block within the group
-          sm100::cp_async16(vst + i * D + c * 8, vg + (bl * 32 + ((en >> 5) & 31)) * D);
-          if (c == 0) sm100::cp_async4(sst + i, sg + bl * 32 + (en & 31));
+          // a listed row lies inside the sequence and the split
+          if (saga_in_bounds(gb0 + bl < blk1 && (gb0 + bl) * 32 + ((en >> 5) & 31) < L, p.err)) {
+            sm100::cp_async16(vst + i * D + c * 8, vg + (bl * 32 + ((en >> 5) & 31)) * D);
+            if (c == 0) sm100::cp_async4(sst + i, sg + bl * 32 + (en & 31));
+          }
         }
       }
       nst += n;

@@ -413,7 +413,8 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
 #pragma unroll
           for (int a = 0; a < kN; ++a) {
             const float x = A[a] * p.scale;
-            if (valid && a < G) p.scores_out[row0 + a * p.row_stride + t] = x;
+            if (valid && a < G && saga_in_bounds(t < p.row_stride, p.err))
+              p.scores_out[row0 + a * p.row_stride + t] = x;
             if (p.hist != nullptr) {
               // top byte of the score's order key, one shared atomic per
               // distinct bin in the warp
@@ -474,7 +475,8 @@ saga_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
             if (a >= G) break;
             const uint32_t bl = __ballot_sync(0xffffffffu, (sel >> a) & 1u);
             if (lane == a) mymask = bl;
-            if ((bl >> lane) & 1u) p.lscore[(hrow0 + a * p.nblk) * 32 + __popc(bl & lt_mask)] = A[a];
+            if (((bl >> lane) & 1u) && saga_in_bounds(valid, p.err))   // only real positions are kept
+              p.lscore[(hrow0 + a * p.nblk) * 32 + __popc(bl & lt_mask)] = A[a];
           }
           if (lane < G) p.lmask[hrow0 + lane * p.nblk] = mymask;
         }

@@ -40,6 +40,18 @@ def test_every_declared_symbol_is_exported(lib):
         assert hasattr(lib, n), f"{n} declared in include/ but not exported"
 
 
+def test_checked_build_exports_the_same_symbols():
+    """The bounds-checked variant (build.py --check) is the same library with
+    index checks compiled in: it loads and exports every declared function."""
+    from sparse_decode_attention_step_b200 import build
+    path = build.CHECK_LIB_PATH
+    if not os.path.exists(path):
+        build.build(check=True)
+    checked = ctypes.CDLL(path)
+    for n in declared_functions():
+        assert hasattr(checked, n), f"{n} not exported by the checked build"
+
+
 def test_status_strings(lib):
     for code in range(6):
         assert saga.status_string(code) != "unknown status"
