@@ -109,12 +109,15 @@ void saga_shape_contiguous(saga_shape *s, int32_t B, int32_t h_q, int32_t h_k,
  * invalid. The workspace must be 256-byte aligned, must be passed to
  * saga_workspace_init once after allocation, and must not be used by two
  * calls that run concurrently. It holds the device error word, per-split
- * partial softmax states and, for refresh, one fp32 score row per
- * (sequence, query head).
+ * partial softmax states, the per-head kept lists of the tensor-core step
+ * (a 32-bit mask and 32 fp32 kept scores per 32-position block) and, for
+ * refresh, one fp32 score row per (sequence, query head) with the radix
+ * select's histograms and bucket lists.
  */
 size_t saga_workspace_size(const saga_shape *shape, int32_t N);
 
-/* Zero a newly allocated workspace (asynchronous on `stream`). */
+/* Zero the error and abort words at the head of a newly allocated workspace
+ * (asynchronous on `stream`); nothing else in it needs clearing. */
 saga_status saga_workspace_init(void *ws, size_t ws_bytes, saga_stream_t stream);
 
 /*
