@@ -77,6 +77,23 @@ def test_topn_with_heavy_ties(dtype, d, h_q, h_k, h_v, N):
     run_topn(w, Kh, Vh, lens, N)
 
 
+@pytest.mark.parametrize("N", [1, 777, 32999])
+def test_topn_rows_of_one_score(N):
+    """Every key of a sequence the same row, so every score of a head is the
+    same value: the radix select's top-byte bucket is the whole row (more
+    than its bucket list holds) and so is the 16-bit bucket (more than the
+    on-chip candidates), which takes the select through its passes over the
+    row; the kept set is the first N positions."""
+    cap = 40000
+    w = synth.Workload("one_score", synth.BF16, B=2, h_q=4, h_k=1, h_v=2, d=64, l_kv=cap, N=N,
+                       R=1, steps=1, seed=97)
+    lens = np.array([cap, 33000], dtype=np.int32)
+    Kh = synth.cache(w, 0, "K", 1, cap, lens)
+    Vh = synth.cache(w, 0, "V", 2, cap, lens)
+    Kh = np.ascontiguousarray(np.repeat(Kh[:, :, :1], cap, axis=2))
+    run_topn(w, Kh, Vh, lens, N)
+
+
 @pytest.mark.parametrize("name,N", [("llama1b_32k", 1024), ("tiny_f32", 64), ("qwen1p5b_128k", 2048)])
 def test_topn_on_the_workloads(name, N):
     """At the workloads' full sizes: caches filled on the device by the
