@@ -67,7 +67,7 @@ struct GatherParams {
   float *partials;          // [B][h_q][SB][d + kRecPad]
   const int32_t *abort;     // the scan's abort word
   int32_t *err;             // device error word (index checks of the checked build)
-  int32_t B, h_q, h_v, SB;
+  int32_t B, h_q, SB;
   int32_t hpv;              // h_q / h_v: query heads per value head
   int64_t blk_per_split;    // 32-position blocks per split
 };

@@ -216,7 +216,7 @@ saga_status run_step(const saga_shape &s, const Plan &pl, StepParams p, int mode
     g.l_kv = p.l_kv; g.cap = p.cap; g.max_l_kv = p.max_l_kv;
     g.lmask = p.lmask; g.lscore = p.lscore; g.nblk = p.nblk;
     g.partials = p.partials; g.abort = p.abort; g.err = p.err;
-    g.B = s.B; g.h_q = s.h_q; g.h_v = s.h_v; g.SB = pl.SB; g.hpv = s.h_q / s.h_v;
+    g.B = s.B; g.h_q = s.h_q; g.SB = pl.SB; g.hpv = s.h_q / s.h_v;
     g.blk_per_split = pl.blk_per_split;
     if ((e = launch_gather(g, s.d, st)) != cudaSuccess) return cuda_fail(e, "gather kernel");
   }
